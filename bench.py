@@ -1,0 +1,533 @@
+"""Benchmark of the quantised linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one call of the layer (rotation of x, load of the packed weight,
+in-register/shared-memory dequantisation, contraction, fp16 store).  The
+default workload is the decode gate/up-projection GEMV (M=1, K=2560, N=9728,
+int4 codes, fp16 scale/zero per 128).  Inputs are seeded and synthetic.
+
+Timing: W warm-up steps, then exactly K steps replayed from CUDA graphs that
+rotate over enough copies of the packed weight to exceed twice the L2 cache,
+bracketed by a barrier and a device synchronisation, measured with CUDA events
+on the launching stream; the max over ranks is reported.  Under torchrun every
+rank runs an independent replica of the workload (the layer is run on one GPU;
+ranks do not exchange data).  ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "µs/call and achieved HBM GB/s (fraction of ~8 TB/s) for quantised GEMV, M=1"
+L2_BYTES = 126 * 1024 * 1024
+
+WORKLOADS = {
+    # name: (description, kind, params)
+    "gateup": ("decode gate/up-proj GEMV: M=1, K=2560, N=9728, int4 g128 fp16 scale/zero, block-128 RHT", "gemv",
+               dict(fn="gateup", M=1)),
+    "tiny": ("tiny linear: M=1, K=256, N=512, int4 g128, block-128 RHT", "gemv", dict(fn="tiny", M=1)),
+    "down1": ("decode down-proj GEMV: M=1, K=9728, N=2560, int3 g128, block-128 RHT", "gemv", dict(fn="down", M=1)),
+    "down4": ("decode down-proj GEMV: M=4, K=9728, N=2560, int3 g128, block-128 RHT", "gemv", dict(fn="down", M=4)),
+    "down16": ("decode down-proj GEMV: M=16, K=9728, N=2560, int3 g128, block-128 RHT", "gemv",
+               dict(fn="down", M=16)),
+    "stack": ("36-layer int6 g128 decoder linear stack + int8 lm_head, M=1 (253 GEMVs per step)", "stack", {}),
+    "prefill256": ("prefill dequant-GEMM: M=256, K=2560, N=9728, mixed int6/int8 64-row blocks, block-128 RHT",
+                   "gemm", dict(M=256)),
+    "prefill1024": ("prefill dequant-GEMM: M=1024, K=2560, N=9728, mixed int6/int8 64-row blocks, block-128 RHT",
+                    "gemm", dict(M=1024)),
+    "prefill2048": ("prefill dequant-GEMM: M=2048, K=2560, N=9728, mixed int6/int8 64-row blocks, block-128 RHT",
+                    "gemm", dict(M=2048)),
+}
+
+
+# --------------------------------------------------------------------------- utils
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "dequant_gemv_packed_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(f.encode())
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    h.update(open(os.path.join(ROOT, "include", "qlin.h"), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str, kernel_hash: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(workload)
+    if not d or d.get("kernel_hash") != kernel_hash:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.lines = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 5:
+                time.sleep(0.01)
+        except FileNotFoundError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.06)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, dist.get_rank(), world, local
+    return None, 0, 1, 0
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(dist, v: float) -> float:
+    if dist is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------- workloads
+
+class Case:
+    """Device-resident inputs of one workload: C rotating copies of the weight."""
+
+    def __init__(self, name: str, copies: int | None = None):
+        from dequant_gemv_packed_b200 import qlin as Q
+        from dequant_gemv_packed_b200 import workloads as W
+        self.Q, self.name = Q, name
+        desc, kind, p = WORKLOADS[name]
+        self.desc_text, self.kind = desc, kind
+        dev = "cuda"
+        if kind == "stack":
+            self.layers = []
+            self.bytes = 0
+            self.flops = 0
+            for _, w, a in W.stack(device=dev):
+                d = Q.Desc.of(w)
+                packed = Q.qlin_pack(d, w.codes)
+                del w.codes
+                ws = torch.empty(max(Q.qlin_gemv_workspace_bytes(1, w.K), 16), dtype=torch.uint8, device=dev)
+                y = torch.empty(1, w.N, dtype=torch.float16, device=dev)
+                self.layers.append((d, packed, w.scales, w.zeros, a.sign_bits, a.x, y, ws))
+                self.bytes += Q.algorithmic_bytes(d)
+                self.flops += 2 * w.N * w.K
+            self.M, self.N, self.K, self.copies = 1, None, None, 1
+            self.weight_bytes_total = self.bytes
+            self.host_sample = None
+            torch.cuda.synchronize()
+            return
+        if kind == "gemv":
+            fn = getattr(W, p["fn"])
+            w, a = fn(device=dev, M=p["M"]) if p["fn"] != "tiny" else fn(device=dev)
+        else:
+            w, a = W.prefill(M=p["M"], device=dev)
+        self.M, self.N, self.K = a.x.shape[0], w.N, w.K
+        self.bits, self.block_bits = w.bits, w.block_bits
+        self.d = Q.Desc.of(w)
+        self.bytes = Q.algorithmic_bytes(self.d)
+        self.flops = 2 * self.M * self.N * self.K
+        packed = Q.qlin_pack(self.d, w.codes)
+        if copies is None:
+            copies = max(1, math.ceil(2 * L2_BYTES / self.bytes) + 1)
+        self.copies = copies
+        self.w = []
+        for c in range(copies):
+            self.w.append((packed.clone(), w.scales.clone(), w.zeros.clone()))
+        self.weight_bytes_total = copies * self.bytes
+        self.sign_bits, self.x = a.sign_bits, a.x
+        self.y = [torch.empty(self.M, self.N, dtype=torch.float16, device=dev) for _ in range(copies)]
+        ws_fn = Q.qlin_gemv_workspace_bytes if kind == "gemv" else Q.qlin_gemm_workspace_bytes
+        self.ws = torch.empty(max(ws_fn(self.M, self.K), 16), dtype=torch.uint8, device=dev)
+        self.call = Q.qlin_gemv if kind == "gemv" else Q.qlin_gemm
+        # host copies for the oracle baseline (packed bytes as the oracle reads them)
+        self.host_sample = (w.codes.cpu().numpy(), w.scales.cpu().numpy(), w.zeros.cpu().numpy(),
+                            a.x.cpu().numpy(), a.sign_bits.cpu().numpy().view(np.uint32))
+        del w
+        torch.cuda.synchronize()
+
+    def launches_per_step(self) -> int:
+        from dequant_gemv_packed_b200 import qlin as Q
+        n = Q.kernel_launches_per_call(self.kind, self.M, self.K)
+        return n * (len(self.layers) if self.kind == "stack" else 1)
+
+    def step(self, i: int):
+        Q = self.Q
+        if self.kind == "stack":
+            for (d, packed, s, z, sb, x, y, ws) in self.layers:
+                Q.qlin_gemv(d, packed, s, z, sb, x, y, ws)
+            return
+        packed, s, z = self.w[i % self.copies]
+        self.call(self.d, packed, s, z, self.sign_bits, self.x, self.y[i % self.copies], self.ws)
+
+
+def time_steps(case: Case, K: int, W: int, dist, stream, graph_len: int = 1024):
+    """Warm up W steps, then time exactly K steps replayed from CUDA graphs."""
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            case.step(i)
+    torch.cuda.synchronize()
+    R = min(graph_len, K) if case.kind != "stack" else 1
+    R = max(R, 1)
+    graphs = []
+    with torch.cuda.stream(stream):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(R):
+                case.step(i)
+        graphs.append((g, R))
+        rem = K % R
+        if rem:
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2, stream=stream):
+                for i in range(rem):
+                    case.step(R + i)
+            graphs.append((g2, rem))
+        # one untimed replay of each graph (uploads the graph)
+        for g_, _ in graphs:
+            g_.replay()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    with sampler:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(K // R):
+                graphs[0][0].replay()
+            if len(graphs) > 1:
+                graphs[1][0].replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+    barrier(dist)
+    ms = start.elapsed_time(end)
+    del graphs
+    return max_over_ranks(dist, ms), sampler.summary()
+
+
+def time_e2e(case: Case, K: int, W: int, stream):
+    """Through the public binding, eager: per step copy x in from pinned host
+    memory, run the layer, copy y back to pinned host memory."""
+    if case.kind == "stack":
+        return None
+    n = min(K, 2000)
+    xh = case.x.cpu().pin_memory()
+    yh = torch.empty(case.M, case.N, dtype=torch.float16).pin_memory()
+    xd = torch.empty_like(case.x)
+    Q = case.Q
+    with torch.cuda.stream(stream):
+        def one(i):
+            packed, s, z = case.w[i % case.copies]
+            xd.copy_(xh, non_blocking=True)
+            case.call(case.d, packed, s, z, case.sign_bits, xd, case.y[i % case.copies], case.ws)
+            yh.copy_(case.y[i % case.copies], non_blocking=True)
+        for i in range(min(W, 50)):
+            one(i)
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(n):
+            one(i)
+        end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / n
+    return {"value": case.bytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "us_per_call": ms * 1e3,
+            "h2d_bytes_per_step": xh.numel() * 2, "d2h_bytes_per_step": yh.numel() * 2,
+            "steps": n, "mode": "eager calls through the Python binding"}
+
+
+def time_cublas(case: Case, stream, reps: int = 2000):
+    """bf16 torch.nn.functional.linear (cuBLAS) of the same shape, same rotation."""
+    if case.kind == "stack":
+        return None
+    copies = max(1, math.ceil(2 * L2_BYTES / (case.N * case.K * 2)) + 1)
+    ws = [torch.randn(case.N, case.K, device="cuda", dtype=torch.bfloat16) for _ in range(copies)]
+    x = case.x.to(torch.bfloat16)
+    with torch.cuda.stream(stream):
+        for i in range(10):
+            torch.nn.functional.linear(x, ws[i % copies])
+        g = torch.cuda.CUDAGraph()
+        R = min(reps, 256)
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(R):
+                torch.nn.functional.linear(x, ws[i % copies])
+        g.replay()
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(1, reps // R)
+        start.record(stream)
+        for _ in range(n):
+            g.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    us = start.elapsed_time(end) * 1e3 / (n * R)
+    del g, ws
+    return us
+
+
+def oracle_step(case_host, rows, bits, block_bits):
+    """One oracle evaluation of the layer restricted to `rows` (from packed bytes)."""
+    from oracle import qlin_oracle as O
+    codes, s, z, x, sb = case_host
+    N, K = codes.shape
+    packed = case_host_packed(case_host, bits, block_bits)
+    c = O.unpack(packed, N, K, bits or None, None if bits else block_bits, rows=rows)
+    return O.linear64(x, c, s[rows], z[rows], sb)
+
+
+_PACKED_CACHE = {}
+
+
+def case_host_packed(case_host, bits, block_bits):
+    key = id(case_host)
+    if key not in _PACKED_CACHE:
+        from oracle import qlin_oracle as O
+        _PACKED_CACHE[key] = O.pack(case_host[0], bits or None, None if bits else block_bits)
+    return _PACKED_CACHE[key]
+
+
+def cpu_oracle_rate(case: Case, budget_s: float = 12.0, rows_per_step: int | None = None):
+    """Oracle throughput (GB/s of the layer's algorithmic bytes) on a bounded
+    sample of the workload's weight rows, BLAS limited to one thread."""
+    from threadpoolctl import threadpool_limits
+    from oracle import qlin_oracle as O
+    codes = case.host_sample[0]
+    N, K = codes.shape
+    bb = None if case.bits else np.asarray(case.block_bits)
+    case_host_packed(case.host_sample, case.bits, bb)
+    per_row = O.algorithmic_bytes(N, K, case.bits or None, bb) / N
+    rng = np.random.default_rng(0)
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        rows = np.sort(rng.choice(N, size=min(64, N), replace=False))
+        oracle_step(case.host_sample, rows, case.bits, bb)
+        t_row = (time.perf_counter() - t0) / len(rows)
+        if rows_per_step is None:
+            rows_per_step = int(max(16, min(N, budget_s / max(t_row, 1e-9))))
+        done_rows, t = 0, 0.0
+        while t < budget_s and done_rows < 4 * N:
+            rows = np.sort(rng.choice(N, size=min(rows_per_step, N), replace=False))
+            t1 = time.perf_counter()
+            oracle_step(case.host_sample, rows, case.bits, bb)
+            t += time.perf_counter() - t1
+            done_rows += len(rows)
+            if rows_per_step is not None and t > 0 and done_rows >= rows_per_step:
+                break
+    gbs = done_rows * per_row / t / 1e9
+    return gbs, done_rows, t
+
+
+# ------------------------------------------------------------------------ main
+
+def run_ours(args):
+    dist, rank, world, local = dist_setup()
+    torch.cuda.set_device(local)
+    from dequant_gemv_packed_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(dist)
+    case = Case(args.workload)
+    stream = torch.cuda.Stream()
+    ms, clocks = time_steps(case, args.steps, args.warmup, dist, stream)
+    ms_step = ms / args.steps
+    peaks = measured_peaks()
+    value = world * case.bytes * args.steps / (ms * 1e-3) / 1e9
+    per_gpu_gbs = case.bytes / (ms_step * 1e-3) / 1e9
+    khash = kernel_source_hash()
+    if case.kind == "gemm":
+        achieved = case.flops / (ms_step * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "peak_source": f"{peaks['source']} dense bf16 cuBLAS burst (fp16 nominal ratio 1:1)"}
+    else:
+        roof = {"bound": "hbm", "achieved": per_gpu_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": per_gpu_gbs / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} HBM copy bandwidth"}
+    roof["traffic"] = ncu_traffic(args.workload, khash)
+    roof["algorithmic_bytes_per_launch"] = case.bytes
+    e2e = time_e2e(case, args.steps, args.warmup, stream)
+    cublas_us = time_cublas(case, stream) if rank == 0 else None
+    cpu = None
+    if rank == 0 and world == 1 and case.host_sample is not None and not args.no_cpu_baseline:
+        gbs, rows, t = cpu_oracle_rate(case, budget_s=args.cpu_budget)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{rows} of {case.N} weight rows (unpack + fp64 dequant + explicit-H rotation + fp64 "
+                         f"matmul), {t:.1f} s, BLAS limited to 1 thread"}
+    if rank == 0:
+        us = ms_step * 1e3
+        cfg = {"workload": case.desc_text, "M": case.M, "K": case.K, "N": case.N,
+               "group": 128, "copies": case.copies,
+               "l2": f"rotating {case.copies} weight copies ({case.weight_bytes_total / 1e6:.0f} MB > 2x L2)"
+               if case.kind != "stack" else f"stack weights {case.weight_bytes_total / 1e9:.2f} GB > L2",
+               "parallelism": f"replicas x{world}", "accumulate": "fp32", "kernel_hash": khash}
+        out = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+               "warmup": args.warmup, "ms_per_step": ms_step, "us_per_call": us,
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+               "data": "synthetic", "config": cfg, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+               "gpu_launches": case.launches_per_step() * args.steps, "clocks": clocks}
+        if cublas_us is not None:
+            out["cublas_bf16"] = {"us_per_call": cublas_us, "speedup": cublas_us / us}
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: rank 0 only, bounded sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from dequant_gemv_packed_b200 import workloads as W
+    from oracle import qlin_oracle as O
+    from threadpoolctl import threadpool_limits
+    desc, kind, p = WORKLOADS[args.workload]
+    if kind == "stack":
+        print(json.dumps({"impl": "reference", "unavailable": "stack workload is not sampled by the CPU oracle arm"}))
+        return
+    if kind == "gemv":
+        fn = getattr(W, p["fn"])
+        w, a = fn(M=p["M"]) if p["fn"] != "tiny" else fn()
+    else:
+        w, a = W.prefill(M=p["M"])
+    N, K = w.N, w.K
+    bb = None if w.bits else w.block_bits.numpy()
+    codes, s, z = w.codes.numpy(), w.scales.numpy(), w.zeros.numpy()
+    x, sb = a.x.numpy(), a.sign_bits.numpy().view(np.uint32)
+    packed = O.pack(codes, w.bits or None, bb)
+    per_row = O.algorithmic_bytes(N, K, w.bits or None, bb) / N
+    rng = np.random.default_rng(0)
+    total_budget = float(os.environ.get("QLIN_REFERENCE_BUDGET_S", "90"))
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        r = np.sort(rng.choice(N, size=min(32, N), replace=False))
+        O.linear64(x, O.unpack(packed, N, K, w.bits or None, bb, rows=r), s[r], z[r], sb)
+        t_row = (time.perf_counter() - t0) / len(r)
+        rows_per_step = int(max(4, min(N, total_budget / max(args.steps + args.warmup, 1) / t_row)))
+        def step():
+            r = np.sort(rng.choice(N, size=rows_per_step, replace=False))
+            O.linear64(x, O.unpack(packed, N, K, w.bits or None, bb, rows=r), s[r], z[r], sb)
+        for _ in range(args.warmup):
+            step()
+        t1 = time.perf_counter()
+        for _ in range(args.steps):
+            step()
+        t = time.perf_counter() - t1
+    ms_step = t * 1e3 / args.steps
+    value = rows_per_step * per_row * args.steps / t / 1e9
+    sample = f"{rows_per_step} of {N} weight rows per step (unpack + fp64 dequant + explicit-H rotation + fp64 matmul)"
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": desc, "M": a.x.shape[0], "K": K, "N": N, "group": 128},
+           "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--workload", default="gateup", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

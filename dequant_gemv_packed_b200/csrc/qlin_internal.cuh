@@ -1,0 +1,107 @@
+// Internal declarations and device routines shared by the qlin kernels.
+//
+// Every kernel that reads packed codes goes through the decode routines here
+// (code_at / dequant_exact / row_of), so qlin_unpack and qlin_dequant exercise
+// exactly the arithmetic that qlin_gemv and qlin_gemm use.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qlin.h"
+
+namespace qlin {
+
+constexpr int kGroup = 128;      // codes per scale/zero group along K
+constexpr int kBlockRows = 64;   // rows per width block in the mixed format
+constexpr int kHadamard = 128;   // block of the activation rotation
+// 1/sqrt(128) = 2^-3.5, rounded to fp32 (0x3DB504F3).
+constexpr float kInvSqrt128 = 0.0883883476483184405f;
+
+// Device view of a packed weight.
+struct PackedView {
+  const uint8_t* codes;      // code stream
+  const uint32_t* start16;   // mixed: block start in 16-byte units [N/64 + 1]
+  const uint8_t* widths;     // mixed: block widths [N/64]
+  int64_t row_bytes_uniform; // uniform: K * bits / 8
+  int32_t N, K;
+  int32_t bits;              // uniform width, 0 = mixed
+};
+
+// Host-side helpers (qlin_api.cu).
+size_t code_bytes(const qlin_desc* d);
+size_t table_offset(const qlin_desc* d);
+PackedView make_view(const qlin_desc* d, const void* packed);
+qlin_status record_cuda(cudaError_t e);
+
+// Launchers (each returns QLIN_OK or QLIN_ERR_CUDA).
+qlin_status launch_pack(const PackedView& v, const uint8_t* codes, uint8_t* packed,
+                        cudaStream_t s);
+qlin_status launch_unpack(const PackedView& v, uint8_t* codes, cudaStream_t s);
+qlin_status launch_dequant(const PackedView& v, const __half* scales, const __half* zeros,
+                           __half* w, cudaStream_t s);
+qlin_status launch_rht(const __half* x, __half* xr, const uint32_t* sign_bits, int M, int K,
+                       cudaStream_t s);
+size_t gemv_workspace_bytes(int M, int K);
+qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half* zeros,
+                        const uint32_t* sign_bits, const __half* x, __half* y, int M,
+                        void* workspace, cudaStream_t s);
+size_t gemm_workspace_bytes(int M, int K);
+qlin_status launch_gemm(const PackedView& v, const __half* scales, const __half* zeros,
+                        const uint32_t* sign_bits, const __half* x, __half* y, int M,
+                        void* workspace, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// Device decode routines
+// ---------------------------------------------------------------------------
+
+// Width of row n and the first 32-bit word of its bit stream.
+__device__ __forceinline__ const uint32_t* row_of(const PackedView& v, int n, int& b) {
+  if (v.bits) {
+    b = v.bits;
+    return reinterpret_cast<const uint32_t*>(v.codes + (size_t)n * (size_t)v.row_bytes_uniform);
+  }
+  const int j = n >> 6;
+  b = v.widths[j];
+  const size_t off = (size_t)v.start16[j] * 16u + (size_t)(n & 63) * (size_t)v.K * b / 8u;
+  return reinterpret_cast<const uint32_t*>(v.codes + off);
+}
+
+// Code k of a row stream of width b: stream bits [b*k, b*k + b).
+__device__ __forceinline__ uint32_t code_at(const uint32_t* row, int b, int k) {
+  const uint32_t bit = (uint32_t)b * (uint32_t)k;
+  const uint32_t w = bit >> 5, sh = bit & 31u;
+  uint32_t q = row[w] >> sh;
+  if (sh + (uint32_t)b > 32u) q |= row[w + 1] << (32u - sh);
+  return q & ((1u << b) - 1u);
+}
+
+// fp16 weight: t = fp32(q) - z, p = s * t (each rounded to nearest in fp32, no
+// fused multiply-add), then one round-to-nearest-even to fp16.
+__device__ __forceinline__ __half dequant_exact(uint32_t q, float s, float z) {
+  const float t = __fsub_rn(__uint2float_rn(q), z);
+  const float p = __fmul_rn(s, t);
+  return __float2half_rn(p);
+}
+
+// Unnormalised 128-point Walsh-Hadamard transform of one block held by a warp:
+// lane l holds elements 4l..4l+3 in v[0..3].  Stages on index bits 0 and 1 run
+// in registers, stages on bits 2..6 exchange with lane l ^ 1, ..., l ^ 16.
+__device__ __forceinline__ void fwht128_warp(float v[4], int lane) {
+  float a0 = v[0] + v[1], a1 = v[0] - v[1];
+  float a2 = v[2] + v[3], a3 = v[2] - v[3];
+  v[0] = a0 + a2; v[2] = a0 - a2;
+  v[1] = a1 + a3; v[3] = a1 - a3;
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float p = __shfl_xor_sync(0xffffffffu, v[i], m);
+      v[i] = upper ? (p - v[i]) : (v[i] + p);
+    }
+  }
+}
+
+}  // namespace qlin

@@ -1,0 +1,192 @@
+/*
+ * qlin.h -- weight-only-quantised linear layer for NVIDIA B200 (sm_100a).
+ *
+ * Computes  Y = rht(X) . dequant(Wq)^T  with fp16 inputs, fp32 accumulation and
+ * fp16 output, where
+ *
+ *   dequant:  w[n][k] = s[n][k/128] * (q[n][k] - z[n][k/128])
+ *             integer codes q of 3, 4, 6 or 8 bits with one fp16 scale s and one
+ *             fp16 zero point z per group of 128 codes along the reduction
+ *             dimension K ("24B0978-Week01-Track2_20-Submission01", section
+ *             "How these techniques accelerate inference on CUDA", paragraph
+ *             "Group-wise affine integer quantisation"; 6- and 8-bit codes:
+ *             "24B0978-Week02-Track2-40-Submission01", section "Recipe").
+ *
+ *   rht:      random Hadamard transform of the activations: per block of 128
+ *             along K, flip the sign of x[k] where sign bit k is set, apply the
+ *             Walsh-Hadamard transform (7 add/subtract butterfly stages) and
+ *             multiply by 1/sqrt(128), so the transform is orthonormal
+ *             ("24B0978-Week01-Track2_20-Submission01", same section, paragraph
+ *             "Random Hadamard transform").
+ *
+ * ---------------------------------------------------------------------------
+ * Packed code layout (the format written by qlin_pack and read by every other
+ * entry point)
+ * ---------------------------------------------------------------------------
+ *   Rows are stored one after the other with no padding.  Row n holds K codes
+ *   of b_n bits as a little-endian bit stream: code k occupies stream bits
+ *   [b_n*k, b_n*k + b_n), least significant bit first, and stream bit j is bit
+ *   (j mod 32) of the little-endian 32-bit word j/32 of the row.
+ *   Example (b = 4): codes 0,1,...,7 form the word 0x76543210.
+ *   A group of 128 codes occupies exactly 16*b bytes (4*b words), so with
+ *   K % 128 == 0 every group, and every row, starts on a 16-byte boundary.
+ *
+ *   Uniform width (desc.bits in {3,4,6,8}): b_n = bits, row n starts at byte
+ *   n*K*bits/8, and the buffer holds N*K*bits/8 bytes.
+ *
+ *   Mixed width (desc.bits == 0): rows come in blocks of 64; block j has width
+ *   block_bits[j] (3, 4, 6 or 8) for all of its rows and all of K
+ *   ("25M2111-Week02-Track2-40-Submission01", section "Method, selection, and
+ *   reproduction": 64-row blocks with per-block byte selectors).  Block j starts
+ *   at byte 8*K*sum_{i<j} block_bits[i]; its row r at 8*K*... + r*K*b_j/8.
+ *   After the code bytes (C = 8*K*sum_j block_bits[j]) the buffer holds a block
+ *   table used by the kernels:
+ *       uint32  start16[N/64 + 1]  at byte C:   block j starts at byte 16*start16[j]
+ *       uint8   width[N/64]        after it:    block_bits[j]
+ *   qlin_packed_bytes() includes the table (rounded up to 16 bytes).
+ *
+ *   Scales and zeros are not repacked: they stay two separate fp16 arrays
+ *   [N][K/128], row-major, passed to every call that dequantises.
+ *
+ *   Sign bits: uint32 [K/32]; bit (k mod 32) of word k/32 set means x[k] is
+ *   negated before the Hadamard transform.
+ *
+ * ---------------------------------------------------------------------------
+ * Conventions
+ * ---------------------------------------------------------------------------
+ *   * Every buffer argument is a DEVICE pointer, allocated and owned by the
+ *     caller, 16-byte aligned, and not aliasing any other argument; the library
+ *     never allocates device memory.  The descriptor (and desc->block_bits) is
+ *     HOST memory, read during the call only.
+ *   * fp16 buffers are passed as uint16_t (IEEE binary16 bit patterns).
+ *   * Calls are asynchronous on `stream` (NULL = the legacy default stream) and
+ *     never synchronise, except qlin_pack on a mixed-width descriptor, which
+ *     copies the block table from pageable host memory (the CUDA runtime
+ *     orders such a copy after the work already queued on the stream).
+ *   * Errors: argument validation happens before any launch and returns a
+ *     negative qlin_status with nothing enqueued; a failed launch returns
+ *     QLIN_ERR_CUDA (the CUDA error is then available from
+ *     qlin_last_cuda_error()).  No C++ exception crosses this interface.
+ *   * Results do not depend on the stream or on previous calls, except that
+ *     qlin_gemv and qlin_gemm overwrite their workspace.
+ */
+#ifndef QLIN_H
+#define QLIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* qlin_stream_t;
+
+typedef enum {
+  QLIN_OK = 0,
+  QLIN_ERR_INVALID_ARG = -1, /* null pointer or inconsistent descriptor            */
+  QLIN_ERR_UNSUPPORTED = -2, /* code width not in {3,4,6,8} (or 0 for mixed)       */
+  QLIN_ERR_SHAPE = -3,       /* K % 128 != 0, N < 1, M out of range, N % 64 (mixed)*/
+  QLIN_ERR_ALIGNMENT = -4,   /* a buffer is not 16-byte aligned                    */
+  QLIN_ERR_CUDA = -5,        /* a CUDA runtime call or kernel launch failed        */
+  QLIN_ERR_WORKSPACE = -6    /* workspace missing or smaller than required         */
+} qlin_status;
+
+/* Describes one packed weight matrix Wq of N output rows and K codes per row.
+ * Plain data, owned by the caller. */
+typedef struct {
+  int32_t N;                  /* output features, >= 1 (mixed: multiple of 64)   */
+  int32_t K;                  /* input features, multiple of 128                 */
+  int32_t bits;               /* 3, 4, 6 or 8; 0 selects mixed widths            */
+  const uint8_t* block_bits;  /* HOST [N/64] widths in {3,4,6,8} when bits == 0,
+                                 else ignored (may be NULL)                       */
+} qlin_desc;
+
+/* Human-readable name of a status code (static storage). */
+const char* qlin_status_string(qlin_status status);
+
+/* The cudaError_t (as int) of the last failed CUDA call made by this library
+ * on the calling thread, 0 if none. */
+int qlin_last_cuda_error(void);
+
+/* Bytes of the packed buffer for `desc` (codes, plus the block table for mixed
+ * widths), a multiple of 16.  Returns 0 for an invalid descriptor. */
+size_t qlin_packed_bytes(const qlin_desc* desc);
+
+/* Bytes of the code stream alone (the layout above without the block table). */
+size_t qlin_code_bytes(const qlin_desc* desc);
+
+/* Pack integer codes into the layout above.
+ *   codes  : device uint8 [N][K], row-major; only the low b_n bits of each code
+ *            of row n are used.
+ *   packed : device, qlin_packed_bytes(desc) bytes, written entirely.
+ * Definition: "24B0978-Week01-Track2_20-Submission01", "How these techniques
+ * accelerate inference on CUDA" (codes stored per group of 128 along K). */
+qlin_status qlin_pack(const qlin_desc* desc, const uint8_t* codes, void* packed,
+                      qlin_stream_t stream);
+
+/* Inverse of qlin_pack: codes (device uint8 [N][K]) from a packed buffer.
+ * Uses the same device decode routines as qlin_gemv and qlin_gemm. */
+qlin_status qlin_unpack(const qlin_desc* desc, const void* packed, uint8_t* codes,
+                        qlin_stream_t stream);
+
+/* Dequantise to fp16: w[n][k] = fp16_rn( fp32(s) * (fp32(q) - fp32(z)) ), each
+ * fp32 operation rounded to nearest, no fused multiply-add, one rounding to
+ * fp16.  This is the exact fp16 weight qlin_gemm multiplies.
+ *   scales, zeros : device fp16 [N][K/128];  w : device fp16 [N][K].
+ * Definition: "24B0978-Week01-Track2_20-Submission01", paragraph "Group-wise
+ * affine integer quantisation". */
+qlin_status qlin_dequant(const qlin_desc* desc, const void* packed, const uint16_t* scales,
+                         const uint16_t* zeros, uint16_t* w, qlin_stream_t stream);
+
+/* Random Hadamard transform of M rows of K activations.
+ *   x  : device fp16 [M][K];  xr : device fp16 [M][K] (may not alias x);
+ *   sign_bits : device uint32 [K/32].
+ * xr = fp16_rn( (1/sqrt(128)) * H_128 * diag(d) * x ) per block of 128, the
+ * butterflies evaluated in fp32 (so within one fp16 ulp of the exact value,
+ * up to fp32 rounding of intermediate sums).  M >= 1, K % 128 == 0.
+ * Definition: "24B0978-Week01-Track2_20-Submission01", paragraph "Random
+ * Hadamard transform". */
+qlin_status qlin_rht(const uint16_t* x, uint16_t* xr, const uint32_t* sign_bits, int32_t M,
+                     int32_t K, qlin_stream_t stream);
+
+/* Workspace bytes qlin_gemv needs for (M, K); 0 means none (workspace may be
+ * NULL).  Depends only on M and K. */
+size_t qlin_gemv_workspace_bytes(int32_t M, int32_t K);
+
+/* Decode-regime quantised linear layer, 1 <= M <= 16:
+ *   y[m][n] = fp16_rn( sum_k rht(x)[m][k] * w[n][k] ), fp32 accumulation,
+ * with rht(x) rounded to fp16 as qlin_rht does.  Weights are dequantised in
+ * registers and never written to memory; the per-group scale and zero may be
+ * applied to the group's partial sum, sum_k s(q - z)x = s(sum qx - z sum x).
+ *   x : device fp16 [M][K] (not rotated);  y : device fp16 [M][N];
+ *   workspace : device buffer of workspace_bytes >= qlin_gemv_workspace_bytes(M, K)
+ *               bytes (may be NULL when that is 0); overwritten.
+ * Definition: "24B0978-Week01-Track2_20-Submission01", section "How these
+ * techniques accelerate inference on CUDA" (fused in-register dequantisation;
+ * per-group scale on the accumulator; activation rotation at runtime). */
+qlin_status qlin_gemv(const qlin_desc* desc, const void* packed, const uint16_t* scales,
+                      const uint16_t* zeros, const uint32_t* sign_bits, const uint16_t* x,
+                      uint16_t* y, int32_t M, void* workspace, size_t workspace_bytes,
+                      qlin_stream_t stream);
+
+/* Workspace bytes qlin_gemm needs for (M, K) (the rotated activations). */
+size_t qlin_gemm_workspace_bytes(int32_t M, int32_t K);
+
+/* Prefill-regime quantised linear layer, any M >= 1 (built for M >= 64):
+ * same result definition as qlin_gemv, with the weight dequantised exactly as
+ * qlin_dequant does into shared memory and multiplied on the tensor cores
+ * (fp16 operands, fp32 accumulation).
+ *   workspace : device buffer of workspace_bytes >= qlin_gemm_workspace_bytes(M, K)
+ *               bytes; overwritten. */
+qlin_status qlin_gemm(const qlin_desc* desc, const void* packed, const uint16_t* scales,
+                      const uint16_t* zeros, const uint32_t* sign_bits, const uint16_t* x,
+                      uint16_t* y, int32_t M, void* workspace, size_t workspace_bytes,
+                      qlin_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLIN_H */

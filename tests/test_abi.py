@@ -1,0 +1,104 @@
+"""CPU checks of the C ABI: the library builds and loads, exports every function
+``include/qlin.h`` declares, and rejects bad arguments before touching a GPU.
+No compute call is made here."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+from dequant_gemv_packed_b200 import build as B
+from dequant_gemv_packed_b200 import qlin as Q
+from oracle import qlin_oracle as O
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "qlin.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return Q.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qlin_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_expected():
+    assert set(declared_functions()) == set(Q.EXPORTED)
+
+
+def test_every_symbol_exported(lib):
+    nm = subprocess.run(["nm", "-D", "--defined-only", Q.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (qlin_\w+)", nm))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_status_strings(lib):
+    for code, name in Q.STATUS_NAMES.items():
+        assert Q.status_string(code).startswith(name)
+
+
+@pytest.mark.parametrize("bits", [3, 4, 6, 8])
+def test_packed_bytes_matches_oracle(lib, bits):
+    for N, K in ((1, 128), (77, 384), (9728, 2560), (2560, 9728), (151936, 2560)):
+        d = Q.Desc(N, K, bits)
+        code = int(O.row_byte_offsets(N, K, bits=bits)[-1])
+        assert Q.qlin_code_bytes(d) == code
+        assert Q.qlin_packed_bytes(d) == (code + 15) // 16 * 16
+
+
+def test_packed_bytes_mixed(lib):
+    bb = np.array([6, 8, 8, 6, 3, 4], dtype=np.uint8)
+    N, K = 64 * len(bb), 2560
+    d = Q.Desc(N, K, 0, bb)
+    code = int(O.row_byte_offsets(N, K, block_bits=bb)[-1])
+    assert Q.qlin_code_bytes(d) == code
+    nb = len(bb)
+    table = (code + 15) // 16 * 16 + 4 * (nb + 1) + nb
+    assert Q.qlin_packed_bytes(d) == (table + 15) // 16 * 16
+
+
+def test_invalid_descriptors(lib):
+    for args in ((0, 128, 4), (8, 100, 4), (8, 128, 5), (8, 128, 2), (65, 128, 0)):
+        bb = [6] * (args[0] // 64 + 1) if args[2] == 0 else None
+        assert Q.qlin_packed_bytes(Q.Desc(*args, block_bits=bb)) == 0
+    assert Q.qlin_packed_bytes(Q.Desc(64, 128, 0, [5])) == 0
+
+
+def _call_gemv(lib, desc, M, ptr=16, ws=0, wsbytes=0):
+    p = ctypes.c_void_p(ptr) if ptr else None
+    return lib.qlin_gemv(desc.ref(), p, p, p, p, p, p, M, ctypes.c_void_p(ws) if ws else None, wsbytes, None)
+
+
+def test_validation_returns_before_launch(lib):
+    d = Q.Desc(512, 256, 4)
+    assert _call_gemv(lib, d, 1, ptr=0) == -1          # null buffers
+    assert _call_gemv(lib, d, 1, ptr=18) == -4         # misaligned
+    assert _call_gemv(lib, d, 0) == -3                 # M out of range
+    assert _call_gemv(lib, d, 17) == -3
+    assert _call_gemv(lib, Q.Desc(512, 200, 4), 1) == -3
+    assert _call_gemv(lib, Q.Desc(512, 256, 5), 1) == -2
+    need = Q.qlin_gemv_workspace_bytes(1, 256)
+    if need:
+        assert _call_gemv(lib, d, 1, ws=0) == -6
+        assert _call_gemv(lib, d, 1, ws=4096, wsbytes=need - 1) == -6
+    p = ctypes.c_void_p(16)
+    assert lib.qlin_gemm(d.ref(), p, p, p, p, p, p, 64, None, 0, None) == -6
+    assert lib.qlin_gemm(d.ref(), p, p, p, p, p, p, 0, p, 1 << 30, None) == -3
+    assert lib.qlin_rht(p, p, p, 1, 256, None) == -1  # in-place not allowed
+    assert lib.qlin_rht(p, ctypes.c_void_p(32), p, 1, 100, None) == -3
+    assert lib.qlin_pack(Q.Desc(64, 128, 0, [7]).ref(), p, p, None) == -2
+
+
+def test_library_refuses_without_build(tmp_path, monkeypatch):
+    monkeypatch.setattr(Q, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(Q, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        Q.lib()

@@ -1,0 +1,255 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bit-exact: packed bytes, unpacked codes, fp16 dequantised weights.
+RHT: within one fp16 ulp of the rounded fp64 transform.
+Layer outputs: max|y - y_ref| <= 2e-3 max|y_ref| and relative Frobenius error
+<= 1e-3 against the fp64 oracle, for every workload shape (tiny int4, gate/up
+int4, down-proj int3 at M = 1/4/16, the 36-layer int6 stack with the int8
+lm_head, the mixed int6/int8 prefill GEMM at M = 256/1024/2048) plus ragged
+and degenerate shapes.
+"""
+import numpy as np
+import pytest
+import torch
+
+from dequant_gemv_packed_b200 import qlin as Q
+from dequant_gemv_packed_b200 import workloads as W
+from oracle import qlin_oracle as O
+
+from parity import assert_close, host, np_u32, oracle_rows, packed_on_device, sample_rows
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from dequant_gemv_packed_b200 import build
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    Q.lib()
+
+
+def _rand_weight(N, K, bits, seed, block_bits=None):
+    w = W.draw_weight(N, K, bits, seed=seed, block_bits=None if bits else torch.as_tensor(block_bits, dtype=torch.uint8))
+    return w.to(DEV)
+
+
+# ------------------------------------------------------------- bit-exact ------
+
+@pytest.mark.parametrize("bits", [3, 4, 6, 8])
+@pytest.mark.parametrize("N,K", [(77, 384), (1, 128), (130, 2560)])
+def test_pack_unpack_bit_exact(bits, N, K):
+    rng = np.random.default_rng(bits * 1000 + N)
+    codes = rng.integers(0, 256, size=(N, K), dtype=np.uint8)  # high bits must be ignored
+    d = Q.Desc(N, K, bits)
+    packed = Q.qlin_pack(d, torch.from_numpy(codes).to(DEV))
+    ref = O.pack(codes, bits=bits)
+    got = packed.cpu().numpy()
+    assert got[:len(ref)].tobytes() == ref.tobytes()
+    back = Q.qlin_unpack(d, packed).cpu().numpy()
+    assert np.array_equal(back, codes & ((1 << bits) - 1))
+
+
+def test_pack_unpack_mixed_bit_exact():
+    bb = np.array([6, 8, 3, 4, 8, 6], dtype=np.uint8)
+    N, K = 64 * len(bb), 640
+    rng = np.random.default_rng(1)
+    codes = rng.integers(0, 256, size=(N, K), dtype=np.uint8)
+    d = Q.Desc(N, K, 0, bb)
+    packed = Q.qlin_pack(d, torch.from_numpy(codes).to(DEV)).cpu().numpy()
+    ref = O.pack(codes, block_bits=bb)
+    assert packed[:len(ref)].tobytes() == ref.tobytes()
+    # block table: starts (16-byte units) and widths
+    t0 = (len(ref) + 15) // 16 * 16
+    starts = packed[t0:t0 + 4 * (len(bb) + 1)].view(np.uint32)
+    off = O.row_byte_offsets(N, K, block_bits=bb)
+    assert np.array_equal(starts.astype(np.int64) * 16, off[::64])
+    assert np.array_equal(packed[t0 + 4 * (len(bb) + 1):t0 + 4 * (len(bb) + 1) + len(bb)], bb)
+    back = Q.qlin_unpack(d, torch.from_numpy(packed).to(DEV)).cpu().numpy()
+    mask = (1 << np.repeat(bb.astype(np.int64), 64)) - 1
+    assert np.array_equal(back, codes & mask[:, None])
+
+
+@pytest.mark.parametrize("bits", [3, 4, 6, 8, 0])
+def test_dequant_bit_exact(bits):
+    bb = [6, 8, 8, 4] if bits == 0 else None
+    N, K = (256 if bits == 0 else 200), 384
+    w = _rand_weight(N, K, bits, seed=bits + 7, block_bits=bb)
+    d, packed = packed_on_device(w)
+    got = Q.qlin_dequant(d, packed, w.scales, w.zeros).cpu().numpy()
+    ref = O.dequant16(w.codes.cpu().numpy(), w.scales.cpu().numpy(), w.zeros.cpu().numpy())
+    assert got.view(np.uint16).tobytes() == ref.view(np.uint16).tobytes()
+
+
+def test_dequant_bit_exact_adversarial_scales():
+    """Arbitrary fp16 scales and zeros (negative, tiny, large, non-integer)."""
+    rng = np.random.default_rng(3)
+    N, K = 64, 256
+    codes = rng.integers(0, 256, size=(N, K), dtype=np.uint8)
+    s = (rng.standard_normal((N, 2)) * np.exp(rng.uniform(-9, 4, (N, 2)))).astype(np.float16)
+    z = (rng.standard_normal((N, 2)) * 100).astype(np.float16)
+    d = Q.Desc(N, K, 8)
+    packed = Q.qlin_pack(d, torch.from_numpy(codes).to(DEV))
+    got = Q.qlin_dequant(d, packed, torch.from_numpy(s).to(DEV), torch.from_numpy(z).to(DEV)).cpu().numpy()
+    ref = O.dequant16(codes, s, z)
+    assert got.view(np.uint16).tobytes() == ref.view(np.uint16).tobytes()
+
+
+# ------------------------------------------------------------------- rht ------
+
+def _ulp16(v):
+    v = np.abs(v).astype(np.float16)
+    return (np.nextafter(v, np.float16(np.inf)) - v).astype(np.float64)
+
+
+@pytest.mark.parametrize("M,K", [(1, 128), (3, 384), (16, 9728), (257, 2560)])
+def test_rht_within_one_ulp(M, K):
+    a = W.draw_activation(M, K, seed=M)
+    ref = O.rht64(a.x.numpy(), np_u32(a.sign_bits))
+    got = Q.qlin_rht(a.x.to(DEV), a.sign_bits.to(DEV)).float().cpu().numpy()
+    err = np.abs(got - ref)
+    # one fp16 ulp of the exact value; values far below the block's scale may
+    # additionally carry the fp32 rounding of the butterfly sums
+    tol = _ulp16(ref) + 1e-6 * np.abs(a.x.float().numpy()).max()
+    assert (err <= tol).all(), float((err - tol).max())
+
+
+# --------------------------------------------------------------- gemv ---------
+
+def _gemv_case(w, a, rows=None, what=""):
+    d, packed = packed_on_device(w)
+    y = Q.qlin_gemv(d, packed, w.scales, w.zeros, a.sign_bits, a.x)
+    torch.cuda.synchronize()
+    ref = oracle_rows(w, a, rows)
+    got = y if rows is None else y[:, torch.as_tensor(rows, device=y.device)]
+    return assert_close(got, ref, what)
+
+
+def test_gemv_tiny_int4():
+    w, a = W.tiny(device=DEV)
+    _gemv_case(w, a, what="tiny")
+
+
+def test_gemv_gateup_int4_full():
+    w, a = W.gateup(device=DEV)
+    _gemv_case(w, a, what="gateup")
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_gemv_down_int3_full(M):
+    w, a = W.down(M=M, device=DEV)
+    _gemv_case(w, a, what=f"down M={M}")
+
+
+def test_gemv_stack_int6_int8_sampled():
+    """Every linear of the 36-layer stack (int6) and the int8 lm_head, sampled rows."""
+    worst = (0.0, 0.0)
+    for i, (name, w, a) in enumerate(W.stack(device=DEV)):
+        rows = sample_rows(w.N, 24, seed=i)
+        r = _gemv_case(w, a, rows, what=name)
+        worst = tuple(max(p, q) for p, q in zip(worst, r))
+        del w, a
+    print("stack worst rel errors", worst)
+
+
+@pytest.mark.parametrize("bits", [3, 4, 6, 8])
+@pytest.mark.parametrize("N,K,M", [(1, 128, 1), (77, 384, 5), (333, 1280, 16), (64, 9728, 2)])
+def test_gemv_ragged(bits, N, K, M):
+    w = _rand_weight(N, K, bits, seed=N + bits)
+    a = W.draw_activation(M, K, seed=N).to(DEV)
+    _gemv_case(w, a, what=f"b{bits} N{N} K{K} M{M}")
+
+
+def test_gemv_mixed():
+    bb = [6, 8, 4, 3, 8]
+    w = _rand_weight(64 * len(bb), 1280, 0, seed=5, block_bits=bb)
+    for M in (1, 3, 16):
+        a = W.draw_activation(M, 1280, seed=M).to(DEV)
+        _gemv_case(w, a, what=f"mixed M{M}")
+
+
+def test_gemv_integer_special_case():
+    """s = 1, z = 0, signs +1, x = row j of H: y[:, n] = sqrt(128) * q[n, j]."""
+    N, K = 96, 256
+    rng = np.random.default_rng(0)
+    codes = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    H = O.hadamard(128)
+    j = 37
+    x = np.zeros((1, K), np.float16)
+    x[0, :128] = H[j]
+    d = Q.Desc(N, K, 4)
+    packed = Q.qlin_pack(d, torch.from_numpy(codes).to(DEV))
+    ones = torch.ones(N, 2, dtype=torch.float16, device=DEV)
+    zeros = torch.zeros(N, 2, dtype=torch.float16, device=DEV)
+    sb = torch.zeros(K // 32, dtype=torch.int32, device=DEV)
+    y = Q.qlin_gemv(d, packed, ones, zeros, sb, torch.from_numpy(x).to(DEV)).float().cpu().numpy()[0]
+    expect = (np.sqrt(128) * codes[:, j]).astype(np.float16).astype(np.float64)
+    assert np.abs(y - expect).max() <= 2e-3 * np.abs(expect).max()
+
+
+def test_gemv_deterministic_and_stream():
+    w, a = W.gateup(device=DEV)
+    d, packed = packed_on_device(w)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        y1 = Q.qlin_gemv(d, packed, w.scales, w.zeros, a.sign_bits, a.x)
+        y2 = Q.qlin_gemv(d, packed, w.scales, w.zeros, a.sign_bits, a.x)
+    s.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_gemv_rejects_misaligned_and_small_workspace():
+    w, a = W.tiny(device=DEV)
+    d, packed = packed_on_device(w)
+    buf = torch.empty(256 * 2 + 8, dtype=torch.float16, device=DEV)
+    xm = buf[1:1 + 256].view(1, 256)  # 2-byte offset
+    with pytest.raises(Q.QlinError) as e:
+        Q.qlin_gemv(d, packed, w.scales, w.zeros, a.sign_bits, xm)
+    assert e.value.status == -4
+    need = Q.qlin_gemv_workspace_bytes(1, 256)
+    if need:
+        small = torch.empty(need - 16, dtype=torch.uint8, device=DEV)
+        with pytest.raises(Q.QlinError) as e:
+            Q.qlin_gemv(d, packed, w.scales, w.zeros, a.sign_bits, a.x, workspace=small)
+        assert e.value.status == -6
+
+
+# --------------------------------------------------------------- gemm ---------
+
+@pytest.mark.parametrize("M", [256, 1024, 2048])
+def test_gemm_prefill_mixed_sampled(M):
+    w, a = W.prefill(M=M, device=DEV)
+    d, packed = packed_on_device(w)
+    y = Q.qlin_gemm(d, packed, w.scales, w.zeros, a.sign_bits, a.x)
+    torch.cuda.synchronize()
+    rows = sample_rows(w.N, 384, seed=M)
+    ref = oracle_rows(w, a, rows)
+    assert_close(y[:, torch.as_tensor(rows, device=DEV)], ref, f"prefill M={M}")
+    assert torch.isfinite(y.float()).all()
+
+
+@pytest.mark.parametrize("bits", [3, 4, 6, 8, 0])
+@pytest.mark.parametrize("N,K,M", [(77, 384, 1), (64, 256, 65), (200, 1280, 17), (448, 2560, 300)])
+def test_gemm_ragged(bits, N, K, M):
+    if bits == 0:
+        N = (N + 63) // 64 * 64
+        bb = ([6, 8] * 8)[:N // 64]
+    else:
+        bb = None
+    w = _rand_weight(N, K, bits, seed=N + M, block_bits=bb)
+    a = W.draw_activation(M, K, seed=M).to(DEV)
+    d, packed = packed_on_device(w)
+    y = Q.qlin_gemm(d, packed, w.scales, w.zeros, a.sign_bits, a.x)
+    torch.cuda.synchronize()
+    assert_close(y, oracle_rows(w, a), f"gemm b{bits} N{N} K{K} M{M}")
+
+
+def test_gemm_matches_gemv_at_m16():
+    w, a = W.down(M=16, device=DEV)
+    d, packed = packed_on_device(w)
+    y1 = Q.qlin_gemv(d, packed, w.scales, w.zeros, a.sign_bits, a.x).float()
+    y2 = Q.qlin_gemm(d, packed, w.scales, w.zeros, a.sign_bits, a.x).float()
+    ref = oracle_rows(w, a)
+    assert_close(y1, ref, "gemv")
+    assert_close(y2, ref, "gemm")
