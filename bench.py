@@ -193,7 +193,7 @@ class Case:
                 d = Q.Desc.of(w)
                 packed = Q.qlin_pack(d, w.codes)
                 del w.codes
-                ws = torch.empty(max(Q.qlin_gemv_workspace_bytes(1, w.K), 16), dtype=torch.uint8, device=dev)
+                ws = torch.empty(max(Q.qlin_gemv_workspace_bytes(d, 1), 16), dtype=torch.uint8, device=dev)
                 y = torch.empty(1, w.N, dtype=torch.float16, device=dev)
                 self.layers.append((d, packed, w.scales, w.zeros, a.sign_bits, a.x, y, ws))
                 self.bytes += Q.algorithmic_bytes(d)
@@ -224,7 +224,7 @@ class Case:
         self.sign_bits, self.x = a.sign_bits, a.x
         self.y = [torch.empty(self.M, self.N, dtype=torch.float16, device=dev) for _ in range(copies)]
         ws_fn = Q.qlin_gemv_workspace_bytes if kind == "gemv" else Q.qlin_gemm_workspace_bytes
-        self.ws = torch.empty(max(ws_fn(self.M, self.K), 16), dtype=torch.uint8, device=dev)
+        self.ws = torch.empty(max(ws_fn(self.d, self.M), 16), dtype=torch.uint8, device=dev)
         self.call = Q.qlin_gemv if kind == "gemv" else Q.qlin_gemm
         # host copies for the oracle baseline (packed bytes as the oracle reads them)
         self.host_sample = (w.codes.cpu().numpy(), w.scales.cpu().numpy(), w.zeros.cpu().numpy(),
@@ -234,8 +234,9 @@ class Case:
 
     def launches_per_step(self) -> int:
         from dequant_gemv_packed_b200 import qlin as Q
-        n = Q.kernel_launches_per_call(self.kind, self.M, self.K)
-        return n * (len(self.layers) if self.kind == "stack" else 1)
+        if self.kind == "stack":
+            return sum(Q.kernel_launches_per_call("gemv", l[0], 1) for l in self.layers)
+        return Q.kernel_launches_per_call(self.kind, self.d, self.M)
 
     def step(self, i: int):
         Q = self.Q
@@ -432,10 +433,11 @@ def run_ours(args):
                 "frac": per_gpu_gbs / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} HBM copy bandwidth"}
     roof["traffic"] = ncu_traffic(args.workload, khash)
     roof["algorithmic_bytes_per_launch"] = case.bytes
-    e2e = time_e2e(case, args.steps, args.warmup, stream)
-    cublas_us = time_cublas(case, stream) if rank == 0 else None
+    e2e = None if args.no_extras else time_e2e(case, args.steps, args.warmup, stream)
+    cublas_us = time_cublas(case, stream) if rank == 0 and not args.no_extras else None
     cpu = None
-    if rank == 0 and world == 1 and case.host_sample is not None and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and case.host_sample is not None and not args.no_cpu_baseline \
+            and not args.no_extras:
         gbs, rows, t = cpu_oracle_rate(case, budget_s=args.cpu_budget)
         cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": f"{rows} of {case.N} weight rows (unpack + fp64 dequant + explicit-H rotation + fp64 "
@@ -520,6 +522,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="time the layer only (no e2e, cuBLAS or CPU-baseline legs), e.g. under a profiler")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

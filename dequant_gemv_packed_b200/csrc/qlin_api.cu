@@ -166,9 +166,9 @@ static qlin_status check_linear(const qlin_desc* d, const void* packed, const ui
   return QLIN_OK;
 }
 
-size_t qlin_gemv_workspace_bytes(int32_t M, int32_t K) {
-  if (M < 1 || M > 16 || K < kGroup || K % kGroup) return 0;
-  return gemv_workspace_bytes(M, K);
+size_t qlin_gemv_workspace_bytes(const qlin_desc* d, int32_t M) {
+  if (check_desc(d) != QLIN_OK || M < 1 || M > 16) return 0;
+  return gemv_workspace_bytes(d->bits, d->N, d->K, M);
 }
 
 qlin_status qlin_gemv(const qlin_desc* d, const void* packed, const uint16_t* scales,
@@ -178,7 +178,7 @@ qlin_status qlin_gemv(const qlin_desc* d, const void* packed, const uint16_t* sc
   qlin_status r = check_linear(d, packed, scales, zeros, sign_bits, x, y);
   if (r != QLIN_OK) return r;
   if (M < 1 || M > 16) return QLIN_ERR_SHAPE;
-  const size_t ws = gemv_workspace_bytes(M, d->K);
+  const size_t ws = gemv_workspace_bytes(d->bits, d->N, d->K, M);
   if (ws && (!workspace || workspace_bytes < ws)) return QLIN_ERR_WORKSPACE;
   if (ws && !aligned16(workspace)) return QLIN_ERR_ALIGNMENT;
   return launch_gemv(make_view(d, packed), reinterpret_cast<const __half*>(scales),
@@ -187,9 +187,15 @@ qlin_status qlin_gemv(const qlin_desc* d, const void* packed, const uint16_t* sc
                      workspace, reinterpret_cast<cudaStream_t>(st));
 }
 
-size_t qlin_gemm_workspace_bytes(int32_t M, int32_t K) {
-  if (M < 1 || K < kGroup || K % kGroup) return 0;
-  return gemm_workspace_bytes(M, K);
+size_t qlin_gemm_workspace_bytes(const qlin_desc* d, int32_t M) {
+  if (check_desc(d) != QLIN_OK || M < 1) return 0;
+  return gemm_workspace_bytes(M, d->K);
+}
+
+qlin_status qlin_device_error(uint32_t* code) {
+  if (!code) return QLIN_ERR_INVALID_ARG;
+  *code = take_gemv_error();
+  return *code == ~0u ? QLIN_ERR_CUDA : QLIN_OK;
 }
 
 qlin_status qlin_gemm(const qlin_desc* d, const void* packed, const uint16_t* scales,

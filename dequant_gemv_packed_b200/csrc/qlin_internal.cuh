@@ -43,7 +43,8 @@ qlin_status launch_dequant(const PackedView& v, const __half* scales, const __ha
                            __half* w, cudaStream_t s);
 qlin_status launch_rht(const __half* x, __half* xr, const uint32_t* sign_bits, int M, int K,
                        cudaStream_t s);
-size_t gemv_workspace_bytes(int M, int K);
+size_t gemv_workspace_bytes(int bits, int N, int K, int M);
+unsigned take_gemv_error();
 qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half* zeros,
                         const uint32_t* sign_bits, const __half* x, __half* y, int M,
                         void* workspace, cudaStream_t s);

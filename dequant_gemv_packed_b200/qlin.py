@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "QLIN_OK", -1: "QLIN_ERR_INVALID_ARG", -2: "QLIN_ERR_UNSUPPOR
 EXPORTED = (
     "qlin_status_string", "qlin_last_cuda_error", "qlin_packed_bytes", "qlin_code_bytes", "qlin_pack",
     "qlin_unpack", "qlin_dequant", "qlin_rht", "qlin_gemv_workspace_bytes", "qlin_gemv",
-    "qlin_gemm_workspace_bytes", "qlin_gemm",
+    "qlin_gemm_workspace_bytes", "qlin_gemm", "qlin_device_error",
 )
 
 
@@ -82,8 +82,9 @@ def lib() -> ctypes.CDLL:
     L.qlin_unpack.argtypes, L.qlin_unpack.restype = [vp, vp, vp, vp], ctypes.c_int
     L.qlin_dequant.argtypes, L.qlin_dequant.restype = [vp, vp, vp, vp, vp, vp], ctypes.c_int
     L.qlin_rht.argtypes, L.qlin_rht.restype = [vp, vp, vp, i32, i32, vp], ctypes.c_int
-    L.qlin_gemv_workspace_bytes.argtypes, L.qlin_gemv_workspace_bytes.restype = [i32, i32], sz
-    L.qlin_gemm_workspace_bytes.argtypes, L.qlin_gemm_workspace_bytes.restype = [i32, i32], sz
+    L.qlin_gemv_workspace_bytes.argtypes, L.qlin_gemv_workspace_bytes.restype = [vp, i32], sz
+    L.qlin_gemm_workspace_bytes.argtypes, L.qlin_gemm_workspace_bytes.restype = [vp, i32], sz
+    L.qlin_device_error.argtypes, L.qlin_device_error.restype = [ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int
     lin = [vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
     L.qlin_gemv.argtypes, L.qlin_gemv.restype = lin, ctypes.c_int
     L.qlin_gemm.argtypes, L.qlin_gemm.restype = lin, ctypes.c_int
@@ -133,12 +134,19 @@ def qlin_code_bytes(desc: Desc) -> int:
     return int(lib().qlin_code_bytes(desc.ref()))
 
 
-def qlin_gemv_workspace_bytes(M: int, K: int) -> int:
-    return int(lib().qlin_gemv_workspace_bytes(M, K))
+def qlin_gemv_workspace_bytes(desc: Desc, M: int) -> int:
+    return int(lib().qlin_gemv_workspace_bytes(desc.ref(), M))
 
 
-def qlin_gemm_workspace_bytes(M: int, K: int) -> int:
-    return int(lib().qlin_gemm_workspace_bytes(M, K))
+def qlin_gemm_workspace_bytes(desc: Desc, M: int) -> int:
+    return int(lib().qlin_gemm_workspace_bytes(desc.ref(), M))
+
+
+def qlin_device_error() -> int:
+    """Read and clear the device-side error word (0: no bounded wait expired)."""
+    v = ctypes.c_uint32(0)
+    _check(lib().qlin_device_error(ctypes.byref(v)), "qlin_device_error")
+    return int(v.value)
 
 
 def qlin_pack(desc: Desc, codes: torch.Tensor, packed: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
@@ -187,7 +195,7 @@ def _linear(fn, what, ws_fn, desc, packed, scales, zeros, sign_bits, x, y, works
         raise ValueError("x.shape[1] != desc.K")
     if y is None:
         y = _alloc((M, desc.N), torch.float16, x)
-    ws = ws_fn(M, K)
+    ws = ws_fn(desc, M)
     if workspace is None and ws:
         workspace = _alloc((ws,), torch.uint8, x)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
@@ -221,9 +229,9 @@ def algorithmic_bytes(desc: Desc) -> int:
     return qlin_code_bytes(desc) + 4 * desc.N * (desc.K // 128) + sel
 
 
-def kernel_launches_per_call(kind: str, M: int, K: int) -> int:
+def kernel_launches_per_call(kind: str, desc: Desc, M: int) -> int:
     """Kernels one call enqueues: the layer kernel, plus the stand-alone rotation
     kernel whenever the call needs a workspace for the rotated activations."""
     if kind == "gemm":
         return 2
-    return 2 if qlin_gemv_workspace_bytes(M, K) else 1
+    return 2 if qlin_gemv_workspace_bytes(desc, M) else 1

@@ -151,9 +151,9 @@ qlin_status qlin_dequant(const qlin_desc* desc, const void* packed, const uint16
 qlin_status qlin_rht(const uint16_t* x, uint16_t* xr, const uint32_t* sign_bits, int32_t M,
                      int32_t K, qlin_stream_t stream);
 
-/* Workspace bytes qlin_gemv needs for (M, K); 0 means none (workspace may be
- * NULL).  Depends only on M and K. */
-size_t qlin_gemv_workspace_bytes(int32_t M, int32_t K);
+/* Workspace bytes qlin_gemv needs for this weight and M; 0 means none (the
+ * workspace may then be NULL).  Returns 0 for an invalid descriptor or M. */
+size_t qlin_gemv_workspace_bytes(const qlin_desc* desc, int32_t M);
 
 /* Decode-regime quantised linear layer, 1 <= M <= 16:
  *   y[m][n] = fp16_rn( sum_k rht(x)[m][k] * w[n][k] ), fp32 accumulation,
@@ -171,8 +171,9 @@ qlin_status qlin_gemv(const qlin_desc* desc, const void* packed, const uint16_t*
                       uint16_t* y, int32_t M, void* workspace, size_t workspace_bytes,
                       qlin_stream_t stream);
 
-/* Workspace bytes qlin_gemm needs for (M, K) (the rotated activations). */
-size_t qlin_gemm_workspace_bytes(int32_t M, int32_t K);
+/* Workspace bytes qlin_gemm needs for this weight and M (the rotated
+ * activations, M*K fp16, rounded up to 256 bytes). */
+size_t qlin_gemm_workspace_bytes(const qlin_desc* desc, int32_t M);
 
 /* Prefill-regime quantised linear layer, any M >= 1 (built for M >= 64):
  * same result definition as qlin_gemv, with the weight dequantised exactly as
@@ -184,6 +185,12 @@ qlin_status qlin_gemm(const qlin_desc* desc, const void* packed, const uint16_t*
                       const uint16_t* zeros, const uint32_t* sign_bits, const uint16_t* x,
                       uint16_t* y, int32_t M, void* workspace, size_t workspace_bytes,
                       qlin_stream_t stream);
+
+/* Reads and clears the device-side error word (0 = no error).  Kernels that
+ * wait on shared-memory barriers bound every wait; a wait that gives up sets a
+ * bit here instead of hanging (the call's output is then invalid).  Synchronous:
+ * waits for all work already queued on the device. */
+qlin_status qlin_device_error(uint32_t* code);
 
 #ifdef __cplusplus
 }

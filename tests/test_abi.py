@@ -85,10 +85,11 @@ def test_validation_returns_before_launch(lib):
     assert _call_gemv(lib, d, 17) == -3
     assert _call_gemv(lib, Q.Desc(512, 200, 4), 1) == -3
     assert _call_gemv(lib, Q.Desc(512, 256, 5), 1) == -2
-    need = Q.qlin_gemv_workspace_bytes(1, 256)
+    assert Q.qlin_gemv_workspace_bytes(d, 1) == 0  # fused rotation, no workspace
+    need = Q.qlin_gemv_workspace_bytes(d, 4)
     if need:
-        assert _call_gemv(lib, d, 1, ws=0) == -6
-        assert _call_gemv(lib, d, 1, ws=4096, wsbytes=need - 1) == -6
+        assert _call_gemv(lib, d, 4, ws=0) == -6
+        assert _call_gemv(lib, d, 4, ws=4096, wsbytes=need - 1) == -6
     p = ctypes.c_void_p(16)
     assert lib.qlin_gemm(d.ref(), p, p, p, p, p, p, 64, None, 0, None) == -6
     assert lib.qlin_gemm(d.ref(), p, p, p, p, p, p, 0, p, 1 << 30, None) == -3

@@ -207,12 +207,13 @@ def test_gemv_rejects_misaligned_and_small_workspace():
     with pytest.raises(Q.QlinError) as e:
         Q.qlin_gemv(d, packed, w.scales, w.zeros, a.sign_bits, xm)
     assert e.value.status == -4
-    need = Q.qlin_gemv_workspace_bytes(1, 256)
-    if need:
-        small = torch.empty(need - 16, dtype=torch.uint8, device=DEV)
-        with pytest.raises(Q.QlinError) as e:
-            Q.qlin_gemv(d, packed, w.scales, w.zeros, a.sign_bits, a.x, workspace=small)
-        assert e.value.status == -6
+    x4 = W.draw_activation(4, 256).x.to(DEV)
+    need = Q.qlin_gemv_workspace_bytes(d, 4)
+    assert need > 0
+    small = torch.empty(need - 16, dtype=torch.uint8, device=DEV)
+    with pytest.raises(Q.QlinError) as e:
+        Q.qlin_gemv(d, packed, w.scales, w.zeros, a.sign_bits, x4, workspace=small)
+    assert e.value.status == -6
 
 
 # --------------------------------------------------------------- gemm ---------
@@ -253,3 +254,9 @@ def test_gemm_matches_gemv_at_m16():
     ref = oracle_rows(w, a)
     assert_close(y1, ref, "gemv")
     assert_close(y2, ref, "gemm")
+
+
+def test_zz_no_device_errors():
+    """No bounded wait in any kernel gave up during the tests above."""
+    torch.cuda.synchronize()
+    assert Q.qlin_device_error() == 0
