@@ -281,12 +281,14 @@ def time_steps(case: Case, K: int, W: int, dist, stream, graph_len: int = 1024):
     sampler = ClockSampler(torch.cuda.current_device())
     with sampler:
         with torch.cuda.stream(stream):
+            torch.cuda.nvtx.range_push("qlin_timed")
             start.record(stream)
             for _ in range(K // R):
                 graphs[0][0].replay()
             if len(graphs) > 1:
                 graphs[1][0].replay()
             end.record(stream)
+            torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
     barrier(dist)
     ms = start.elapsed_time(end)

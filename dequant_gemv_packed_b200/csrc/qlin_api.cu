@@ -194,8 +194,10 @@ size_t qlin_gemm_workspace_bytes(const qlin_desc* d, int32_t M) {
 
 qlin_status qlin_device_error(uint32_t* code) {
   if (!code) return QLIN_ERR_INVALID_ARG;
-  *code = take_gemv_error();
-  return *code == ~0u ? QLIN_ERR_CUDA : QLIN_OK;
+  const unsigned a = take_gemv_error(), b = take_gemm_error();
+  if (a == ~0u || b == ~0u) return QLIN_ERR_CUDA;
+  *code = a | (b << 8);
+  return QLIN_OK;
 }
 
 qlin_status qlin_gemm(const qlin_desc* d, const void* packed, const uint16_t* scales,

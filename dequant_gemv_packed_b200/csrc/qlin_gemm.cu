@@ -1,74 +1,343 @@
-// qlin_gemm: prefill-regime quantised linear layer.
+// qlin_gemm: prefill-regime quantised linear layer on the 5th-generation tensor
+// cores (tcgen05, accumulators in tensor memory).
 //
-// The activations are rotated into the workspace, the weight is dequantised
-// exactly (fp16, as qlin_dequant) into shared memory tile by tile, and the
-// tiles are multiplied with fp32 accumulation.
+// Y = rht(X) . dequant(W)^T.  The activations are rotated into the workspace
+// by the stand-alone rotation kernel; the weight is dequantised exactly as
+// qlin_dequant does (fp32 subtract and multiply, one rounding to fp16) into
+// shared memory, inside the main loop, and never reaches global memory
+// ("24B0978-Week01-Track2_20-Submission01", "How these techniques accelerate
+// inference on CUDA").
+//
+// Tiling (one CTA per SM, persistent over output tiles):
+//   MMA  D[128 weight rows][BN activation rows] += A[128][64] . B[BN][64]^T
+//   A = dequantised weight rows, K-major, 128-byte swizzle, written by 8
+//       dequantisation warps straight from the packed codes in global memory;
+//   B = rotated activations, K-major, 128-byte swizzle, loaded by TMA;
+//   D = fp32 in tensor memory, two accumulators (2 x 256 columns) so the
+//       epilogue of one tile overlaps the main loop of the next.
+// Warp roles: 0 TMA producer, 1 MMA issuer (one thread) and TMEM owner,
+// 4..7 epilogue (TMEM lane quarters 0..3), 8..15 dequantisation.
+// The weight tile is the MMA's M side because dequantisation costs ALU work
+// per weight element per activation tile: with 256 activation rows per tile
+// each weight element is dequantised once per 256 rows of X.
+#include <cuda.h>
+
+#include <algorithm>
+
 #include "qlin_internal.cuh"
+#include "qlin_sm100.cuh"
 
 namespace qlin {
 
-namespace simt {
-constexpr int BM = 64, BN = 64, BK = 32;
+__device__ unsigned int g_gemm_error;
+
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kBK = 64;        // k per stage: 64 fp16 = one 128-byte swizzle row
+constexpr int kBMw = 128;      // weight rows per tile (MMA M)
+constexpr int kBNmax = 256;    // activation rows per tile (MMA N)
+constexpr int kAStage = kBMw * kBK * 2;     // 16 KB
+constexpr int kBStage = kBNmax * kBK * 2;   // 32 KB
+constexpr int kThreads = 512;
+constexpr int kDeqWarp0 = 8, kDeqWarps = 8;
+constexpr int kEpiWarp0 = 4;
+constexpr int kTmemCols = 512;
+constexpr int kSmemBytes = kStages * (kAStage + kBStage) + 1024 /*barriers*/ + 1024 /*align*/;
+
+struct GemmArgs {
+  PackedView v;
+  const __half* scales;
+  const __half* zeros;
+  __half* y;
+  int M, BN, m_tiles, n_tiles, KB;
+};
+
+__device__ __forceinline__ void gemm_fail(unsigned code) { atomicOr(&g_gemm_error, code); }
+
+__device__ __forceinline__ void wait_or_fail(uint64_t* bar, uint32_t parity, unsigned code) {
+  if (!mbar_wait(bar, parity, &g_gemm_error)) gemm_fail(code);
 }
 
-// 64x64 output tile per CTA, 256 threads, 4x4 outputs per thread.
-__global__ void __launch_bounds__(256) gemm_simt_kernel(PackedView v, const __half* __restrict__ scales,
-                                                        const __half* __restrict__ zeros,
-                                                        const __half* __restrict__ xr,
-                                                        __half* __restrict__ y, int M) {
-  using namespace simt;
-  __shared__ float xs[BK][BM + 1];
-  __shared__ float ws[BK][BN + 1];
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
-  const int tid = threadIdx.x;
-  const int tx = tid % 16, ty = tid / 16;
-  const int G = v.K / kGroup;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < v.K; k0 += BK) {
-    for (int i = tid; i < BM * BK; i += 256) {
-      const int r = i / BK, c = i % BK;
-      const int m = m0 + r;
-      xs[c][r] = m < M ? __half2float(xr[(size_t)m * v.K + k0 + c]) : 0.f;
+// ---- tcgen05 / TMA wrappers ----
+
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  // K-major, 128-byte swizzle: rows of 128 B, 8-row groups 1024 B apart (SBO),
+  // LBO unused (encoded 1), descriptor version 1, layout type 2.
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t dtmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_addr(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// ---- exact dequantisation of 32 consecutive codes of one row ----
+// q -> fp32 exactly via the bit pattern 2^23 + q (0x4B000000 | q) minus 2^23,
+// then t = q - z and p = s * t, each rounded to nearest in fp32, then fp16.
+template <int B>
+__device__ __forceinline__ void dequant32(const uint8_t* src, float s, float z, uint32_t (&out)[16]) {
+  constexpr int kWords = B;  // 32 codes * B bits = B words
+  uint32_t w[kWords + 1];
+  if constexpr (B == 4 || B == 8) {
+    const uint4* p = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+    for (int i = 0; i < kWords / 4; ++i) {
+      const uint4 v = __ldg(p + i);
+      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
     }
-    for (int i = tid; i < BN * BK; i += 256) {
-      const int r = i / BK, c = i % BK;
-      const int n = n0 + r;
-      float w = 0.f;
-      if (n < v.N) {
-        int b;
-        const uint32_t* row = row_of(v, n, b);
-        const int k = k0 + c, g = k / kGroup;
-        w = __half2float(dequant_exact(code_at(row, b, k), __half2float(scales[(size_t)n * G + g]),
-                                       __half2float(zeros[(size_t)n * G + g])));
-      }
-      ws[c][r] = w;
+  } else if constexpr (B == 6) {
+    const uint2* p = reinterpret_cast<const uint2*>(src);
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+      const uint2 v = __ldg(p + i);
+      w[2 * i] = v.x; w[2 * i + 1] = v.y;
     }
-    __syncthreads();
-#pragma unroll 4
-    for (int c = 0; c < BK; ++c) {
-      float a[4], bb[4];
+  } else {
+    const uint32_t* p = reinterpret_cast<const uint32_t*>(src);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = xs[c][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) bb[j] = ws[c][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
-    }
-    __syncthreads();
+    for (int i = 0; i < 3; ++i) w[i] = __ldg(p + i);
   }
+  w[kWords] = 0;
+  constexpr uint32_t kMask = (1u << B) - 1u;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + ty * 4 + i;
-    if (m >= M) continue;
+  for (int i = 0; i < 32; i += 2) {
+    float f[2];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx * 4 + j;
-      if (n < v.N) y[(size_t)m * v.N + n] = __float2half_rn(acc[i][j]);
+    for (int j = 0; j < 2; ++j) {
+      const int bit = B * (i + j);
+      const uint32_t q = __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31) & kMask;
+      const float qf = __fsub_rn(__uint_as_float(0x4B000000u | q), 8388608.0f);
+      f[j] = __fmul_rn(s, __fsub_rn(qf, z));
     }
+    __half2 h = __floats2half2_rn(f[0], f[1]);
+    out[i >> 1] = *reinterpret_cast<uint32_t*>(&h);
   }
 }
+
+__device__ __forceinline__ void dequant32_any(int b, const uint8_t* src, float s, float z, uint32_t (&out)[16]) {
+  switch (b) {
+    case 3: dequant32<3>(src, s, z, out); break;
+    case 4: dequant32<4>(src, s, z, out); break;
+    case 6: dequant32<6>(src, s, z, out); break;
+    default: dequant32<8>(src, s, z, out); break;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                              const __grid_constant__ GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* As = smem;
+  uint8_t* Bs = smem + kStages * kAStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Bs + kStages * kBStage);
+  uint64_t* st_empty = bars;
+  uint64_t* a_full = bars + kStages;
+  uint64_t* b_full = bars + 2 * kStages;
+  uint64_t* acc_full = bars + 3 * kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles = a.m_tiles * a.n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&st_empty[s], 1);
+      mbar_init(&a_full[s], kDeqWarps);
+      mbar_init(&b_full[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      int g = 0;
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int m0 = (t % a.m_tiles) * a.BN;
+        for (int kb = 0; kb < a.KB; ++kb, ++g) {
+          const int s = g % kStages, u = g / kStages;
+          if (u > 0) wait_or_fail(&st_empty[s], (u - 1) & 1, 1u);
+          mbar_arrive_expect_tx(&b_full[s], (uint32_t)a.BN * kBK * 2);
+          tma_load_2d(Bs + s * kBStage, &xmap, kb * kBK, m0, &b_full[s]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      // kind::f16, fp32 accumulate, fp16 A and B, both K-major, M = 128, N = BN.
+      const uint32_t idesc = (1u << 4) | ((uint32_t)(a.BN >> 3) << 17) | ((uint32_t)(kBMw >> 4) << 24);
+      int g = 0, i = 0;
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+        const int abuf = i & 1, ua = i >> 1;
+        if (ua > 0) wait_or_fail(&acc_empty[abuf], (ua - 1) & 1, 2u);
+        tc_fence_after();
+        const uint32_t dtmem = tmem_base + (uint32_t)(abuf * kBNmax);
+        for (int kb = 0; kb < a.KB; ++kb, ++g) {
+          const int s = g % kStages, u = g / kStages;
+          wait_or_fail(&a_full[s], u & 1, 4u);
+          wait_or_fail(&b_full[s], u & 1, 8u);
+          tc_fence_after();
+          const uint64_t ad = umma_desc_sw128(smem_addr(As + s * kAStage));
+          const uint64_t bd = umma_desc_sw128(smem_addr(Bs + s * kBStage));
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)  // 16 fp16 = 32 bytes = 2 descriptor units
+            umma_f16(dtmem, ad + 2u * k, bd + 2u * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&st_empty[s]);
+        }
+        umma_commit(&acc_full[abuf]);
+      }
+    }
+  } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+    // --------------------------------------------------------- epilogue --
+    const int q = warp & 3;  // TMEM lanes 32q..32q+31 = weight rows of the tile
+    int i = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      const int m0 = (t % a.m_tiles) * a.BN;
+      const int n0 = (t / a.m_tiles) * kBMw;
+      const int abuf = i & 1, ua = i >> 1;
+      wait_or_fail(&acc_full[abuf], ua & 1, 16u);
+      tc_fence_after();
+      const int n = n0 + 32 * q + lane;
+      for (int c0 = 0; c0 < a.BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(abuf * kBNmax + c0), r);
+        if (n < a.v.N) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int m = m0 + c0 + j;
+            if (m < a.M) a.y[(size_t)m * a.v.N + n] = __float2half_rn(__uint_as_float(r[j]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[abuf]);
+    }
+  } else if (warp >= kDeqWarp0) {
+    // ---------------------------------------------------- dequantisation --
+    const int dt = threadIdx.x - kDeqWarp0 * 32;  // 0..255
+    const int r = dt >> 1, h = dt & 1;            // tile row, half of the 64-code stage slice
+    const int G = a.v.K / kGroup;
+    int g = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+      const int n = (t / a.m_tiles) * kBMw + r;
+      const bool valid = n < a.v.N;
+      int b = 4;
+      const uint8_t* row = nullptr;
+      if (valid) row = reinterpret_cast<const uint8_t*>(row_of(a.v, n, b));
+      for (int kb = 0; kb < a.KB; ++kb, ++g) {
+        const int s = g % kStages, u = g / kStages;
+        uint32_t out[16];
+        if (valid) {
+          const int k0 = kb * kBK + 32 * h;
+          const size_t gi = (size_t)n * G + (k0 >> 7);
+          dequant32_any(b, row + (size_t)k0 * b / 8, __half2float(a.scales[gi]), __half2float(a.zeros[gi]), out);
+        } else {
+#pragma unroll
+          for (int i2 = 0; i2 < 16; ++i2) out[i2] = 0u;
+        }
+        if (u > 0) wait_or_fail(&st_empty[s], (u - 1) & 1, 32u);
+        uint8_t* arow = As + s * kAStage + r * 128;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = 4 * h + j;
+          *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) =
+              make_uint4(out[4 * j], out[4 * j + 1], out[4 * j + 2], out[4 * j + 3]);
+        }
+        fence_async_shared();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[s]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+}
+
+// ---- host side ----
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+}  // namespace
 
 size_t gemm_workspace_bytes(int M, int K) { return ((size_t)M * K * 2 + 255) & ~(size_t)255; }
 
@@ -78,10 +347,50 @@ qlin_status launch_gemm(const PackedView& v, const __half* scales, const __half*
   __half* xr = static_cast<__half*>(workspace);
   qlin_status r = launch_rht(x, xr, sign_bits, M, v.K, s);
   if (r != QLIN_OK) return r;
-  dim3 grid((v.N + simt::BN - 1) / simt::BN, (M + simt::BM - 1) / simt::BM);
-  if (grid.y > 65535) return QLIN_ERR_SHAPE;
-  gemm_simt_kernel<<<grid, 256, 0, s>>>(v, scales, zeros, xr, y, M);
+
+  GemmArgs a;
+  a.v = v;
+  a.scales = scales;
+  a.zeros = zeros;
+  a.y = y;
+  a.M = M;
+  a.BN = std::min(kBNmax, (M + 15) / 16 * 16);
+  a.m_tiles = (M + a.BN - 1) / a.BN;
+  a.n_tiles = (v.N + kBMw - 1) / kBMw;
+  a.KB = v.K / kBK;
+
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return record_cuda(cudaErrorNotSupported);
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)v.K, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)v.K * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)a.BN};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xr, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return record_cuda(cudaErrorInvalidValue);
+
+  static unsigned long long configured = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record_cuda(e);
+  if (dev >= 64 || !((configured >> dev) & 1ull)) {
+    e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return record_cuda(e);
+    if (dev < 64) configured |= 1ull << dev;
+  }
+  const int tiles = a.m_tiles * a.n_tiles;
+  const int grid = std::min(tiles, 148);
+  gemm_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(map, a);
   return record_cuda(cudaGetLastError());
+}
+
+unsigned take_gemm_error() {
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_gemm_error, sizeof(v)) != cudaSuccess) return ~0u;
+  if (v) cudaMemcpyToSymbol(g_gemm_error, &zero, sizeof(zero));
+  return v;
 }
 
 }  // namespace qlin

@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) gemv1_kernel(const __grid_cons
     if (lane != 0) return;
     for (int t = 0; t < nchunks; ++t) {
       const int s = t % p.stages;
-      if (t >= p.stages && !mbar_wait(&empty[s], ((t / p.stages) - 1) & 1)) gemv_fail(1u);
+      if (t >= p.stages && !mbar_wait(&empty[s], ((t / p.stages) - 1) & 1, &g_gemv_error)) gemv_fail(1u);
       uint8_t* st = smem + (size_t)s * p.stage_bytes;
       __half* ssm = reinterpret_cast<__half*>(st + (size_t)Rc * p.row_stride);
       __half* zsm = ssm + p.sz_halves;
@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) gemv1_kernel(const __grid_cons
   // -------------------------------------------------------- main loop ----
   for (int t = 0; t < nchunks; ++t) {
     const int s = t % p.stages;
-    if (!mbar_wait(&full[s], (t / p.stages) & 1)) gemv_fail(2u);
+    if (!mbar_wait(&full[s], (t / p.stages) & 1, &g_gemv_error)) gemv_fail(2u);
     const uint8_t* st = smem + (size_t)s * p.stage_bytes;
     const __half* ssm = reinterpret_cast<const __half*>(st + (size_t)Rc * p.row_stride);
     const __half* zsm = ssm + p.sz_halves;

@@ -45,6 +45,7 @@ qlin_status launch_rht(const __half* x, __half* xr, const uint32_t* sign_bits, i
                        cudaStream_t s);
 size_t gemv_workspace_bytes(int bits, int N, int K, int M);
 unsigned take_gemv_error();
+unsigned take_gemm_error();
 qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half* zeros,
                         const uint32_t* sign_bits, const __half* x, __half* y, int M,
                         void* workspace, cudaStream_t s);

@@ -16,7 +16,7 @@ from dequant_gemv_packed_b200 import qlin as Q
 from dequant_gemv_packed_b200 import workloads as W
 from oracle import qlin_oracle as O
 
-from parity import assert_close, host, np_u32, oracle_rows, packed_on_device, sample_rows
+from parity import assert_close, assert_close_abs, host, np_u32, oracle_rows, packed_on_device, sample_rows
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -121,6 +121,8 @@ def _gemv_case(w, a, rows=None, what=""):
     d, packed = packed_on_device(w)
     y = Q.qlin_gemv(d, packed, w.scales, w.zeros, a.sign_bits, a.x)
     torch.cuda.synchronize()
+    if w.N < 16:
+        return assert_close_abs(y, w, a, rows, what)
     ref = oracle_rows(w, a, rows)
     got = y if rows is None else y[:, torch.as_tensor(rows, device=y.device)]
     return assert_close(got, ref, what)
@@ -231,7 +233,7 @@ def test_gemm_prefill_mixed_sampled(M):
 
 
 @pytest.mark.parametrize("bits", [3, 4, 6, 8, 0])
-@pytest.mark.parametrize("N,K,M", [(77, 384, 1), (64, 256, 65), (200, 1280, 17), (448, 2560, 300)])
+@pytest.mark.parametrize("N,K,M", [(77, 384, 1), (64, 256, 65), (200, 1280, 17), (448, 2560, 300), (256, 640, 600)])
 def test_gemm_ragged(bits, N, K, M):
     if bits == 0:
         N = (N + 63) // 64 * 64
@@ -244,6 +246,7 @@ def test_gemm_ragged(bits, N, K, M):
     y = Q.qlin_gemm(d, packed, w.scales, w.zeros, a.sign_bits, a.x)
     torch.cuda.synchronize()
     assert_close(y, oracle_rows(w, a), f"gemm b{bits} N{N} K{K} M{M}")
+    assert Q.qlin_device_error() == 0
 
 
 def test_gemm_matches_gemv_at_m16():
