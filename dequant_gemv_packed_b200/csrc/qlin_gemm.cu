@@ -23,6 +23,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "qlin_internal.cuh"
 #include "qlin_sm100.cuh"
@@ -394,3 +395,118 @@ unsigned take_gemm_error() {
 }
 
 }  // namespace qlin
+
+// ---------------------------------------------------------------------------
+// qlin_gemm_noalloc: qlin_gemm with a library-owned scratch buffer.
+//
+// qlin_gemm needs a caller-provided workspace for the rotated activations.
+// Some callers cannot allocate device memory where they run the layer: a plugin
+// hosted by another runtime that owns every device allocation, or a serving loop
+// that forbids allocation once it is running (cudaMalloc may synchronise the
+// device).  This entry point keeps the rotated activations in the file-scope
+// array below instead, so the caller passes only inputs and outputs.
+//
+// * The array holds kNoallocMaxElems fp16 values (16 MiB); every GPU that loads
+//   the library holds it until the process exits.  Calls with M*K above that
+//   limit are rejected with QLIN_ERR_SHAPE before anything is enqueued.
+// * Host code must not hand the array's name to a kernel: on the host it is a
+//   stand-in, not a device address.  The first call on each device, with that
+//   device current, looks up the array's device address once with
+//   cudaGetSymbolAddress and remembers it; make that first call before any
+//   stream capture.
+// * Every call on a device uses the same array and leaves its rotated
+//   activations there.  Each call overwrites the M*K values it reads before
+//   reading them, so nothing needs clearing; calls that overlap on the GPU (two
+//   streams, or two threads) race on the array and must be serialised by the
+//   caller.
+// ---------------------------------------------------------------------------
+
+namespace qlin {
+namespace {
+
+constexpr size_t kNoallocMaxElems = (size_t)8 << 20;  // 8,388,608 fp16 = 16 MiB
+constexpr int kNoallocMaxDevices = 64;
+
+static __device__ __align__(256) uint16_t g_noalloc_rotated_x[kNoallocMaxElems];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once).
+qlin_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record_cuda(e);
+  if (dev < 0 || dev >= kNoallocMaxDevices) return QLIN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_rotated_x);
+    if (e != cudaSuccess) return record_cuda(e);
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return QLIN_OK;
+}
+
+bool noalloc_width_ok(int b) { return b == 3 || b == 4 || b == 6 || b == 8; }
+bool noalloc_aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace qlin
+
+extern "C" qlin_status qlin_gemm_noalloc(const qlin_desc* d, const void* packed, const uint16_t* scales,
+                                         const uint16_t* zeros, const uint32_t* sign_bits, const uint16_t* x,
+                                         uint16_t* y, int32_t M, qlin_stream_t st) {
+  using namespace qlin;
+  if (!d) return QLIN_ERR_INVALID_ARG;
+  if (d->N < 1 || d->K < kGroup || d->K % kGroup || M < 1) return QLIN_ERR_SHAPE;
+  if (d->bits == 0) {
+    if (d->N % kBlockRows) return QLIN_ERR_SHAPE;
+    if (!d->block_bits) return QLIN_ERR_INVALID_ARG;
+    for (int j = 0; j < d->N / kBlockRows; ++j)
+      if (!noalloc_width_ok(d->block_bits[j])) return QLIN_ERR_UNSUPPORTED;
+  } else if (!noalloc_width_ok(d->bits)) {
+    return QLIN_ERR_UNSUPPORTED;
+  }
+  if (!packed || !scales || !zeros || !sign_bits || !x || !y) return QLIN_ERR_INVALID_ARG;
+  if (!noalloc_aligned(packed) || !noalloc_aligned(scales) || !noalloc_aligned(zeros) ||
+      !noalloc_aligned(sign_bits) || !noalloc_aligned(x) || !noalloc_aligned(y))
+    return QLIN_ERR_ALIGNMENT;
+  if ((size_t)M * (size_t)d->K > kNoallocMaxElems) return QLIN_ERR_SHAPE;
+  void* scratch = nullptr;
+  qlin_status r = noalloc_scratch(&scratch);
+  if (r != QLIN_OK) return r;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(st);
+  const PackedView v = make_view(d, packed);
+  __half* xr = static_cast<__half*>(scratch);
+  r = launch_rht(reinterpret_cast<const __half*>(x), xr, sign_bits, M, v.K, s);
+  if (r != QLIN_OK) return r;
+
+  GemmArgs a;
+  a.v = v;
+  a.scales = reinterpret_cast<const __half*>(scales);
+  a.zeros = reinterpret_cast<const __half*>(zeros);
+  a.y = reinterpret_cast<__half*>(y);
+  a.M = M;
+  a.BN = std::min(kBNmax, (M + 15) / 16 * 16);
+  a.m_tiles = (M + a.BN - 1) / a.BN;
+  a.n_tiles = (v.N + kBMw - 1) / kBMw;
+  a.KB = v.K / kBK;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return record_cuda(cudaErrorNotSupported);
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)v.K, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)v.K * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)a.BN};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+      CUDA_SUCCESS)
+    return record_cuda(cudaErrorInvalidValue);
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return record_cuda(e);
+  const int tiles = a.m_tiles * a.n_tiles;
+  gemm_tc_kernel<<<std::min(tiles, 148), kThreads, kSmemBytes, s>>>(map, a);
+  return record_cuda(cudaGetLastError());
+}

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "QLIN_OK", -1: "QLIN_ERR_INVALID_ARG", -2: "QLIN_ERR_UNSUPPOR
 EXPORTED = (
     "qlin_status_string", "qlin_last_cuda_error", "qlin_packed_bytes", "qlin_code_bytes", "qlin_pack",
     "qlin_unpack", "qlin_dequant", "qlin_rht", "qlin_gemv_workspace_bytes", "qlin_gemv",
-    "qlin_gemm_workspace_bytes", "qlin_gemm", "qlin_device_error",
+    "qlin_gemm_workspace_bytes", "qlin_gemm", "qlin_device_error", "qlin_gemm_noalloc",
 )
 
 
@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
     lin = [vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
     L.qlin_gemv.argtypes, L.qlin_gemv.restype = lin, ctypes.c_int
     L.qlin_gemm.argtypes, L.qlin_gemm.restype = lin, ctypes.c_int
+    L.qlin_gemm_noalloc.argtypes, L.qlin_gemm_noalloc.restype = [vp, vp, vp, vp, vp, vp, vp, i32, vp], ctypes.c_int
     _lib = L
     return L
 

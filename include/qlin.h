@@ -186,6 +186,27 @@ qlin_status qlin_gemm(const qlin_desc* desc, const void* packed, const uint16_t*
                       uint16_t* y, int32_t M, void* workspace, size_t workspace_bytes,
                       qlin_stream_t stream);
 
+/* qlin_gemm for callers that cannot allocate device memory: the pages have no
+ * counterpart; this is a library convenience.  qlin_gemm needs a workspace for
+ * the rotated activations, but some callers cannot allocate one where they run
+ * the layer (for example a plugin inside another runtime that owns all device
+ * allocations, or a serving loop that forbids allocation once running, since
+ * cudaMalloc can synchronise the device).  This entry point allocates nothing:
+ * it keeps the rotated activations in a fixed 16 MiB array inside the library
+ * (every GPU that loads the library holds it until the process exits).
+ *   Arguments, layout and result: as qlin_gemm, without the workspace.
+ *   Limit: M * K <= 8,388,608; larger calls return QLIN_ERR_SHAPE and enqueue
+ *   nothing.
+ *   The first call on each device (with that device current) looks up the
+ *   array's device address once; make that first call before any stream
+ *   capture.  All calls on a device share the array and leave their rotated
+ *   activations in it; each call overwrites what it reads, so nothing needs
+ *   clearing, but calls that overlap on the GPU (several streams or threads)
+ *   race on it and must be serialised by the caller. */
+qlin_status qlin_gemm_noalloc(const qlin_desc* desc, const void* packed, const uint16_t* scales,
+                              const uint16_t* zeros, const uint32_t* sign_bits, const uint16_t* x,
+                              uint16_t* y, int32_t M, qlin_stream_t stream);
+
 /* Reads and clears the device-side error word (0 = no error).  Kernels that
  * wait on shared-memory barriers bound every wait; a wait that gives up sets a
  * bit here instead of hanging (the call's output is then invalid).  Synchronous:
