@@ -419,6 +419,16 @@ def run_ours(args):
     barrier(dist)
     case = Case(args.workload)
     stream = torch.cuda.Stream()
+    from dequant_gemv_packed_b200 import qlin as Q
+    overlap = case.kind in ("gemv", "stack") and not args.no_overlap
+    no_overlap = None
+    if overlap:
+        # the same K steps with each call waiting for the previous one to finish
+        Q.qlin_set_overlap(False)
+        ms0, _ = time_steps(case, args.steps, args.warmup, dist, stream)
+        no_overlap = {"ms_per_step": ms0 / args.steps,
+                      "GB/s": case.bytes * args.steps / (ms0 * 1e-3) / 1e9}
+    Q.qlin_set_overlap(overlap)
     ms, clocks = time_steps(case, args.steps, args.warmup, dist, stream)
     ms_step = ms / args.steps
     peaks = measured_peaks()
@@ -450,7 +460,9 @@ def run_ours(args):
                "group": 128, "copies": case.copies,
                "l2": f"rotating {case.copies} weight copies ({case.weight_bytes_total / 1e6:.0f} MB > 2x L2)"
                if case.kind != "stack" else f"stack weights {case.weight_bytes_total / 1e9:.2f} GB > L2",
-               "parallelism": f"replicas x{world}", "accumulate": "fp32", "kernel_hash": khash}
+               "parallelism": f"replicas x{world}", "accumulate": "fp32", "kernel_hash": khash,
+               "launch": ("CUDA graph, consecutive calls overlapped by programmatic dependent launch "
+                          "(qlin_set_overlap(1))") if overlap else "CUDA graph, serial launches"}
         out = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
                "warmup": args.warmup, "ms_per_step": ms_step, "us_per_call": us,
                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
@@ -458,6 +470,8 @@ def run_ours(args):
                "gpu_launches": case.launches_per_step() * args.steps, "clocks": clocks}
         if cublas_us is not None:
             out["cublas_bf16"] = {"us_per_call": cublas_us, "speedup": cublas_us / us}
+        if no_overlap is not None:
+            out["no_overlap"] = no_overlap
         print(json.dumps(out), flush=True)
     if dist is not None:
         dist.destroy_process_group()
@@ -524,6 +538,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-overlap", action="store_true", help="serial launches only (no programmatic dependent launch)")
     ap.add_argument("--no-extras", action="store_true",
                     help="time the layer only (no e2e, cuBLAS or CPU-baseline legs), e.g. under a profiler")
     args = ap.parse_args()

@@ -1,5 +1,6 @@
 // C ABI of the qlin library: argument validation, status codes, dispatch.
 // Nothing here computes the layer; it checks arguments and enqueues kernels.
+#include <atomic>
 #include <cstring>
 #include <vector>
 
@@ -8,6 +9,9 @@
 namespace qlin {
 
 static thread_local int g_last_cuda_error = 0;
+static std::atomic<int> g_overlap{0};
+
+bool overlap_enabled() { return g_overlap.load(std::memory_order_relaxed) != 0; }
 
 qlin_status record_cuda(cudaError_t e) {
   if (e == cudaSuccess) return QLIN_OK;
@@ -87,6 +91,8 @@ const char* qlin_status_string(qlin_status s) {
 }
 
 int qlin_last_cuda_error(void) { return g_last_cuda_error; }
+
+int qlin_set_overlap(int enable) { return g_overlap.exchange(enable ? 1 : 0); }
 
 size_t qlin_packed_bytes(const qlin_desc* d) {
   return check_desc(d) == QLIN_OK ? packed_bytes(d) : 0;

@@ -44,7 +44,15 @@ constexpr int kThreads = 512;
 constexpr int kDeqWarp0 = 8, kDeqWarps = 8;
 constexpr int kEpiWarp0 = 4;
 constexpr int kTmemCols = 512;
-constexpr int kSmemBytes = kStages * (kAStage + kBStage) + 1024 /*barriers*/ + 1024 /*align*/;
+// Codes of one 128-code group of the whole 128-row weight tile (two MMA
+// stages), copied cooperatively and coalesced by the dequantisation threads
+// into a ring of kCodeRing slots: row r at r * 128 bytes, its 16-byte piece c
+// at slot (c ^ (r & 7)) (bank-conflict-free reads of the row slices).
+constexpr int kDeqThreads = kDeqWarps * 32;
+constexpr int kCodeRing = 2;
+constexpr int kCodeSlotBytes = kBMw * 128;
+constexpr int kSmemBytes = kStages * (kAStage + kBStage) + kCodeRing * kCodeSlotBytes + 1024 /*barriers*/ +
+                           1024 /*align*/;
 
 struct GemmArgs {
   PackedView v;
@@ -116,55 +124,96 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 
 __device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// ---- exact dequantisation of 32 consecutive codes of one row ----
-// q -> fp32 exactly via the bit pattern 2^23 + q (0x4B000000 | q) minus 2^23,
-// then t = q - z and p = s * t, each rounded to nearest in fp32, then fp16.
+// ---- cp.async (per-thread asynchronous copies into shared memory) ----
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// ---- packed fp32 pairs (each lane of the pair rounded as its scalar op) ----
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// ---- exact dequantisation of 32 consecutive codes of one row (from shared memory) ----
+// q -> fp32 exactly through the bit pattern 2^23 + q (0x4B000000 | q) minus
+// 2^23; then t = q - z and p = s * t, each rounded to nearest in fp32 (the same
+// operations as dequant_exact, two lanes per instruction), then fp16.
 template <int B>
-__device__ __forceinline__ void dequant32(const uint8_t* src, float s, float z, uint32_t (&out)[16]) {
-  constexpr int kWords = B;  // 32 codes * B bits = B words
-  uint32_t w[kWords + 1];
-  if constexpr (B == 4 || B == 8) {
-    const uint4* p = reinterpret_cast<const uint4*>(src);
+__device__ __forceinline__ void dequant32(const uint8_t* row, int r, int o, float s, float z, uint32_t (&out)[16]) {
+  // row: this row's 128-byte slot line; o: byte offset of the 32 codes in the row
+  uint32_t w[B + 1];
+  const int sw = r & 7;
+  if constexpr (B == 8 || B == 4) {
 #pragma unroll
-    for (int i = 0; i < kWords / 4; ++i) {
-      const uint4 v = __ldg(p + i);
+    for (int i = 0; i < B / 4; ++i) {
+      const uint4 v = *reinterpret_cast<const uint4*>(row + ((((o >> 4) + i) ^ sw) << 4));
       w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
     }
   } else if constexpr (B == 6) {
-    const uint2* p = reinterpret_cast<const uint2*>(src);
 #pragma unroll
     for (int i = 0; i < 3; ++i) {
-      const uint2 v = __ldg(p + i);
+      const int oo = o + 8 * i;
+      const uint2 v = *reinterpret_cast<const uint2*>(row + (((oo >> 4) ^ sw) << 4) + (oo & 15));
       w[2 * i] = v.x; w[2 * i + 1] = v.y;
     }
   } else {
-    const uint32_t* p = reinterpret_cast<const uint32_t*>(src);
 #pragma unroll
-    for (int i = 0; i < 3; ++i) w[i] = __ldg(p + i);
+    for (int i = 0; i < 3; ++i) {
+      const int oo = o + 4 * i;
+      w[i] = *reinterpret_cast<const uint32_t*>(row + (((oo >> 4) ^ sw) << 4) + (oo & 15));
+    }
   }
-  w[kWords] = 0;
+  w[B] = 0;
   constexpr uint32_t kMask = (1u << B) - 1u;
+  const uint64_t c23 = pk2(8388608.0f, 8388608.0f), zz = pk2(z, z), ss = pk2(s, s);
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
-    float f[2];
+    uint32_t m[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      const int bit = B * (i + j);
-      const uint32_t q = __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31) & kMask;
-      const float qf = __fsub_rn(__uint_as_float(0x4B000000u | q), 8388608.0f);
-      f[j] = __fmul_rn(s, __fsub_rn(qf, z));
+      const int c = i + j;
+      if constexpr (B == 8) {
+        m[j] = __byte_perm(w[c >> 2], 0x4B000000u, 0x7540u | (uint32_t)(c & 3));
+      } else {
+        const int bit = B * c;
+        const uint32_t v = ((bit & 31) + B <= 32) ? (w[bit >> 5] >> (bit & 31))
+                                                  : __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31);
+        m[j] = (v & kMask) | 0x4B000000u;
+      }
     }
-    __half2 h = __floats2half2_rn(f[0], f[1]);
+    const uint64_t t = sub2(sub2(pk2(__uint_as_float(m[0]), __uint_as_float(m[1])), c23), zz);
+    float p0, p1;
+    upk2(mul2(ss, t), p0, p1);
+    __half2 h = __floats2half2_rn(p0, p1);
     out[i >> 1] = *reinterpret_cast<uint32_t*>(&h);
   }
 }
 
-__device__ __forceinline__ void dequant32_any(int b, const uint8_t* src, float s, float z, uint32_t (&out)[16]) {
+__device__ __forceinline__ void dequant32_any(int b, const uint8_t* row, int r, int o, float s, float z,
+                                              uint32_t (&out)[16]) {
   switch (b) {
-    case 3: dequant32<3>(src, s, z, out); break;
-    case 4: dequant32<4>(src, s, z, out); break;
-    case 6: dequant32<6>(src, s, z, out); break;
-    default: dequant32<8>(src, s, z, out); break;
+    case 3: dequant32<3>(row, r, o, s, z, out); break;
+    case 4: dequant32<4>(row, r, o, s, z, out); break;
+    case 6: dequant32<6>(row, r, o, s, z, out); break;
+    default: dequant32<8>(row, r, o, s, z, out); break;
   }
 }
 
@@ -174,7 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* As = smem;
   uint8_t* Bs = smem + kStages * kAStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Bs + kStages * kBStage);
+  uint8_t* Cs = Bs + kStages * kBStage;  // code ring
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Cs + kCodeRing * kCodeSlotBytes);
   uint64_t* st_empty = bars;
   uint64_t* a_full = bars + kStages;
   uint64_t* b_full = bars + 2 * kStages;
@@ -276,40 +326,95 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     }
   } else if (warp >= kDeqWarp0) {
     // ---------------------------------------------------- dequantisation --
+    // Per 128-code group of the tile, all 256 threads copy the tile's codes
+    // (16-byte pieces, consecutive threads on consecutive pieces of a row) one
+    // group ahead into the code ring, then thread (r, h) dequantises row r,
+    // codes [32h, 32h + 32) of each of the group's two 64-code MMA stages.
     const int dt = threadIdx.x - kDeqWarp0 * 32;  // 0..255
-    const int r = dt >> 1, h = dt & 1;            // tile row, half of the 64-code stage slice
+    const int r = dt >> 1, h = dt & 1;
     const int G = a.v.K / kGroup;
-    int g = 0;
+    // copy cursor: tile ct, group cg
+    int ct = blockIdx.x, cg = 0;
+    const uint8_t* cbase[2] = {nullptr, nullptr};
+    int cb[2] = {4, 4}, cvalid = 0;
+    auto copy_tile = [&]() {
+      if (ct >= tiles) return;
+      const int n0 = (ct / a.m_tiles) * kBMw;
+      cvalid = min(kBMw, a.v.N - n0);
+      for (int hh = 0; hh < 2; ++hh)
+        if (64 * hh < cvalid) cbase[hh] = reinterpret_cast<const uint8_t*>(row_of(a.v, n0 + 64 * hh, cb[hh]));
+    };
+    auto issue_group = [&](int slot) {
+      if (ct < tiles) {
+        uint8_t* dst = Cs + slot * kCodeSlotBytes;
+        const int P0 = 64 * cb[0], P = P0 + (cvalid > 64 ? 64 * cb[1] : 0);
+        for (int i = dt; i < P; i += kDeqThreads) {
+          const int hh = i >= P0 ? 1 : 0;
+          const int ii = i - hh * P0, bb = cb[hh];
+          const int rr = ii / bb, c = ii - rr * bb;
+          const int row = 64 * hh + rr;
+          if (row < cvalid) {
+            const uint8_t* src = cbase[hh] + (size_t)rr * (size_t)(a.v.K / 8 * bb) + (size_t)cg * 16 * bb + 16 * c;
+            cp_async16(dst + row * 128 + ((c ^ (row & 7)) << 4), src);
+          }
+        }
+        if (++cg == G) {
+          cg = 0;
+          ct += gridDim.x;
+          copy_tile();
+        }
+      }
+      cp_async_commit();
+    };
+    copy_tile();
+    issue_group(0);
+    int q = 0, g = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int n = (t / a.m_tiles) * kBMw + r;
       const bool valid = n < a.v.N;
       int b = 4;
-      const uint8_t* row = nullptr;
-      if (valid) row = reinterpret_cast<const uint8_t*>(row_of(a.v, n, b));
-      for (int kb = 0; kb < a.KB; ++kb, ++g) {
-        const int s = g % kStages, u = g / kStages;
-        uint32_t out[16];
-        if (valid) {
-          const int k0 = kb * kBK + 32 * h;
-          const size_t gi = (size_t)n * G + (k0 >> 7);
-          dequant32_any(b, row + (size_t)k0 * b / 8, __half2float(a.scales[gi]), __half2float(a.zeros[gi]), out);
-        } else {
-#pragma unroll
-          for (int i2 = 0; i2 < 16; ++i2) out[i2] = 0u;
+      if (valid) (void)row_of(a.v, n, b);
+      const __half* srow = a.scales + (size_t)n * G;
+      const __half* zrow = a.zeros + (size_t)n * G;
+      float sc = valid ? __half2float(srow[0]) : 0.f, zc = valid ? __half2float(zrow[0]) : 0.f;
+      for (int gi = 0; gi < G; ++gi, ++q) {
+        // next group's scale and zero (loaded now, used one group later)
+        float sn = 0.f, zn = 0.f;
+        if (valid && gi + 1 < G) {
+          sn = __half2float(srow[gi + 1]);
+          zn = __half2float(zrow[gi + 1]);
         }
-        if (u > 0) wait_or_fail(&st_empty[s], (u - 1) & 1, 32u);
-        uint8_t* arow = As + s * kAStage + r * 128;
+        cp_async_wait<0>();            // this thread's copies of group q have landed
+        named_barrier(2, kDeqThreads);  // everyone's have; everyone is done with group q - 1
+        issue_group((q + 1) % kCodeRing);
+        const uint8_t* crow = Cs + (q % kCodeRing) * kCodeSlotBytes + r * 128;
+#pragma unroll 1
+        for (int j = 0; j < 2; ++j, ++g) {
+          const int s = g % kStages, u = g / kStages;
+          uint32_t out[16];
+          if (valid) {
+            dequant32_any(b, crow, r, (8 * j + 4 * h) * b, sc, zc, out);
+          } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int c = 4 * h + j;
-          *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) =
-              make_uint4(out[4 * j], out[4 * j + 1], out[4 * j + 2], out[4 * j + 3]);
+            for (int i2 = 0; i2 < 16; ++i2) out[i2] = 0u;
+          }
+          if (u > 0) wait_or_fail(&st_empty[s], (u - 1) & 1, 32u);
+          uint8_t* arow = As + s * kAStage + r * 128;
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const int c = 4 * h + jj;
+            *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) =
+                make_uint4(out[4 * jj], out[4 * jj + 1], out[4 * jj + 2], out[4 * jj + 3]);
+          }
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[s]);
         }
-        fence_async_shared();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[s]);
+        sc = sn;
+        zc = zn;
       }
     }
+    cp_async_wait<0>();
   }
 
   tc_fence_before();

@@ -20,15 +20,24 @@
 //   * Each consumer lane then owns one fixed "unit" of K (64 codes for int4 and
 //     int6, 128 for int3, 32 for int8) and keeps its slice of rotated x in
 //     registers for the whole kernel, walking down the rows of each chunk.
-//   * Codes are turned into fp16 without conversions: masking a code into the
-//     mantissa of the fp16 constant 1024 (0x6400) gives exactly 1024 + c*q,
-//     where c is a power of two fixed by the code's bit position; one lop3 (or
-//     prmt) produces two such values.  They are multiplied with x in fp16 x
+//   * 4- and 8-bit codes: the lane converts its rotated x to 16-bit integers
+//     with one power-of-two scale per unit (exact for values within 2^4 of the
+//     unit's largest magnitude, else rounded at 2^-14 of it) and takes
+//     sum_k q_k x_k exactly in int32 with dp2a (two 16x8-bit products per
+//     instruction); nibbles are spread to byte lanes with one mask each.
+//   * 3- and 6-bit codes are turned into fp16 without conversions: masking a
+//     code into the mantissa of the fp16 constant 1024 (0x6400) gives exactly
+//     1024 + c*q, where c is a power of two fixed by the code's bit position;
+//     one lop3 produces two such values.  They are multiplied with x in fp16 x
 //     fp16 -> fp32 fused multiply-adds, one accumulator per position scale c,
 //     and the constant part 1024*sum(x/c) is removed afterwards with a
 //     correction computed once per lane from its x registers.
 //   * Per (row, unit) the lane stores s*(sum q x - z*sum x) to shared memory;
 //     rows are summed over units in a fixed order (deterministic results).
+//   * With qlin_set_overlap(1) the kernel is launched as a programmatic
+//     dependent: it lets the next kernel start launching at once, streams its
+//     weight before waiting on the previous kernel, and waits only before it
+//     reads x (so back-to-back calls overlap their ramp and drain).
 // Other cases (M > 1, mixed widths): the activation rotation runs as its own
 // kernel into the workspace, then gemv_simple_kernel.
 #include <algorithm>
@@ -45,7 +54,11 @@ namespace {
 constexpr uint32_t kMagic = 0x64006400u;  // fp16 1024.0 in both halves
 constexpr int kMaxConsumerWarps = 16;
 constexpr int kMaxThreads = (kMaxConsumerWarps + 1) * 32;
-constexpr int kSmemLimit = 227 * 1024;
+// Two CTAs per SM: at most 10 consumer warps each, so registers stay <= 93.
+constexpr int kMaxConsumerWarps2 = 10;
+constexpr int kMaxThreads2 = (kMaxConsumerWarps2 + 1) * 32;
+constexpr int kSmemLimit = 227 * 1024;      // one CTA per SM
+constexpr int kSmemLimit2 = 113 * 1024;     // two CTAs per SM
 constexpr int kChunkTarget = 24 * 1024;
 constexpr int kPartialBudget = 48 * 1024;
 constexpr int kMaxStages = 16;
@@ -63,7 +76,9 @@ struct Plan {
   int U;               // units per row
   int UW, RS, NW;      // units per warp, row slots per warp, consumer warps
   int rows_per_cta, grid;
-  int row_bytes, row_stride;
+  int row_bytes, row_stride;  // row_stride == row_bytes: a chunk is one contiguous copy
+  int swap_odd;        // 32-byte units: lanes on odd row slots read their two halves swapped
+  int ctas_per_sm;
   int rows_per_chunk;  // R_c, a multiple of RS
   int stages;
   int chunks_per_window;
@@ -89,46 +104,57 @@ struct Args {
 // Each returns sum_k (1024/c_k + q_k) * x_k over the unit, where c_k is the
 // position scale of code k; the lane subtracts corr = sum_k 1024/c_k * x_k.
 
-__device__ __forceinline__ float dot_unit(const uint32_t (&w)[8], const uint32_t (&x)[32],
-                                          int_<4>) {
-  float a1a = 0.f, a1b = 0.f, a16a = 0.f, a16b = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t wi = w[i], w8 = wi >> 8;
-    const uint32_t t0 = (wi & 0x000F000Fu) | kMagic;  // (q0, q4)
-    const uint32_t t1 = (wi & 0x00F000F0u) | kMagic;  // (16 q1, 16 q5)
-    const uint32_t t2 = (w8 & 0x000F000Fu) | kMagic;  // (q2, q6)
-    const uint32_t t3 = (w8 & 0x00F000F0u) | kMagic;  // (16 q3, 16 q7)
-    const uint32_t x01 = x[4 * i], x23 = x[4 * i + 1], x45 = x[4 * i + 2], x67 = x[4 * i + 3];
-    float& A1 = (i & 1) ? a1b : a1a;
-    float& A16 = (i & 1) ? a16b : a16a;
-    A1 = fma_f16f32(lo16(t0), lo16(x01), A1);
-    A16 = fma_f16f32(lo16(t1), hi16(x01), A16);
-    A1 = fma_f16f32(lo16(t2), lo16(x23), A1);
-    A16 = fma_f16f32(lo16(t3), hi16(x23), A16);
-    A1 = fma_f16f32(hi16(t0), lo16(x45), A1);
-    A16 = fma_f16f32(hi16(t1), hi16(x45), A16);
-    A1 = fma_f16f32(hi16(t2), lo16(x67), A1);
-    A16 = fma_f16f32(hi16(t3), hi16(x67), A16);
-  }
-  return (a1a + a1b) + 0.0625f * (a16a + a16b);
+// Integer decoders (4- and 8-bit codes): dp2a multiplies two signed 16-bit
+// activations by two unsigned 8-bit codes and adds to an int32, exactly.
+// The lane's x registers hold 16-bit integer pairs ordered to match the byte
+// lanes below.
+__device__ __forceinline__ int dp2a_lo(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
-__device__ __forceinline__ float dot_unit(const uint32_t (&w)[8], const uint32_t (&x)[16],
-                                          int_<8>) {
-  float aa = 0.f, ab = 0.f;
+// int4: word i holds codes 8i..8i+7.  x pairs: (x0,x2) (x4,x6) (x1,x3) (x5,x7).
+__device__ __forceinline__ int dot_unit_int(const uint32_t (&w)[8], const uint32_t (&x)[32], int_<4>) {
+  int a0 = 0, a1 = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t p0 = __byte_perm(w[i], 0x64646464u, 0x4240);  // (q0, q2)
-    const uint32_t p1 = __byte_perm(w[i], 0x64646464u, 0x4341);  // (q1, q3)
-    const uint32_t x01 = x[2 * i], x23 = x[2 * i + 1];
-    float& A = (i & 1) ? ab : aa;
-    A = fma_f16f32(lo16(p0), lo16(x01), A);
-    A = fma_f16f32(lo16(p1), hi16(x01), A);
-    A = fma_f16f32(hi16(p0), lo16(x23), A);
-    A = fma_f16f32(hi16(p1), hi16(x23), A);
+    const uint32_t lo = w[i] & 0x0F0F0F0Fu;         // q0 q2 q4 q6
+    const uint32_t hi = (w[i] >> 4) & 0x0F0F0F0Fu;  // q1 q3 q5 q7
+    int& A = (i & 1) ? a1 : a0;
+    A = dp2a_lo(x[4 * i], lo, A);
+    A = dp2a_hi(x[4 * i + 1], lo, A);
+    A = dp2a_lo(x[4 * i + 2], hi, A);
+    A = dp2a_hi(x[4 * i + 3], hi, A);
   }
-  return aa + ab;
+  return a0 + a1;
+}
+
+// int8: word i holds codes 4i..4i+3.  x pairs: (x0,x1) (x2,x3).
+__device__ __forceinline__ int dot_unit_int(const uint32_t (&w)[8], const uint32_t (&x)[16], int_<8>) {
+  int a0 = 0, a1 = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int& A = (i & 1) ? a1 : a0;
+    A = dp2a_lo(x[2 * i], w[i], A);
+    A = dp2a_hi(x[2 * i + 1], w[i], A);
+  }
+  return a0 + a1;
+}
+
+// Position of code c (0-based within the unit) in the lane's int16 x layout.
+template <int B>
+__device__ __forceinline__ int int_slot(int c) {
+  if (B == 8) return c;  // natural order
+  // int4: word i = c/8, code j = c%8 -> pair order (0,2) (4,6) (1,3) (5,7)
+  const int i = c >> 3, j = c & 7;
+  const int pair = ((j & 1) << 1) | (j >> 2);  // j=0,2 ->0; 4,6 ->1; 1,3 ->2; 5,7 ->3
+  return 8 * i + 2 * pair + ((j >> 1) & 1);
 }
 
 // 48 bits of a 48-byte unit starting at bit 48*p: A = bits [0, 32), B = bits [32, 48) (+ junk above).
@@ -234,10 +260,36 @@ __device__ __forceinline__ float corr_weight(int i) {
 
 __device__ __forceinline__ void gemv_fail(unsigned code) { atomicOr(&g_gemv_error, code); }
 
+// sum_k q_k x_k over one unit: exact integer dot (scaled back) or the fp16
+// mantissa-code path minus its constant part.
+template <int B, bool kInt, int kWords, int kXw>
+__device__ __forceinline__ float unit_dot(const uint32_t (&w)[kWords], const uint32_t (&x)[kXw], float corr,
+                                          float xinv) {
+  if constexpr (kInt) {
+    return (float)dot_unit_int(w, x, int_<B>()) * xinv;
+  } else {
+    return dot_unit(w, x, int_<B>()) - corr;
+  }
+}
+
+template <int kWords>
+__device__ __forceinline__ void load_unit(const uint8_t* src, uint32_t (&w)[kWords], int half_first = 0) {
+  const uint4* cp = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int i = 0; i < kWords / 4; ++i) {
+    const uint4 v = cp[kWords == 8 ? (i ^ half_first) : i];
+    w[4 * i] = v.x;
+    w[4 * i + 1] = v.y;
+    w[4 * i + 2] = v.z;
+    w[4 * i + 3] = v.w;
+  }
+}
+
 // ------------------------------------------------------------------ kernel --
 
 template <int B>
-__global__ void __launch_bounds__(kMaxThreads, 1) gemv1_kernel(const __grid_constant__ Args a) {
+__global__ void __launch_bounds__(B == 3 ? kMaxThreads : kMaxThreads2, B == 3 ? 1 : 2)
+    gemv1_kernel(const __grid_constant__ Args a) {
   using UT = UnitT<B>;
   constexpr int kWords = UT::kBytes / 4;
   constexpr int kXw = UT::kCodes / 2;  // half2 registers of x per lane
@@ -263,6 +315,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1) gemv1_kernel(const __grid_cons
     mbar_fence_init();
   }
   __syncthreads();
+  // Programmatic dependent launch: the next kernel on the stream may start
+  // launching now; this kernel's own weight stream does not depend on the
+  // previous kernel, x and y do (grid_dependency_wait below).
+  if (tid == 0) grid_launch_dependents();
 
   if (warp == p.NW) {
     // ------------------------------------------------------- producer ----
@@ -282,9 +338,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) gemv1_kernel(const __grid_cons
       }
       const uint32_t szb = bl > al ? (uint32_t)(bl - al) * 2u : 0u;
       mbar_arrive_expect_tx(&full[s], (uint32_t)cr * p.row_bytes + 2u * szb);
-      const uint8_t* src = a.codes + (size_t)(n0 + cr0) * p.row_bytes;
-      for (int r = 0; r < cr; ++r)
-        bulk_g2s(st + (size_t)r * p.row_stride, src + (size_t)r * p.row_bytes, p.row_bytes, &full[s]);
+      bulk_g2s(st, a.codes + (size_t)(n0 + cr0) * p.row_bytes, (uint32_t)cr * p.row_bytes, &full[s]);
       if (szb) {
         bulk_g2s(ssm, a.scales + al, szb, &full[s]);
         bulk_g2s(zsm, a.zeros + al, szb, &full[s]);
@@ -295,24 +349,38 @@ __global__ void __launch_bounds__(kMaxThreads, 1) gemv1_kernel(const __grid_cons
 
   // --------------------------------------------------------- prologue ----
   // Rotate x into shared memory: warp per block of 128, lane holds 4 values.
+  // All of a warp's x loads are issued before any is used (one memory latency).
+  grid_dependency_wait();
   const int nblk = a.K / kHadamard;
-  for (int blk = warp; blk < nblk; blk += p.NW) {
-    const int k0 = blk * kHadamard + 4 * lane;
-    const uint2 raw = *reinterpret_cast<const uint2*>(a.x + k0);
-    const uint32_t sw = a.sign_bits[blk * 4 + (lane >> 3)] >> (4 * (lane & 7));
-    const __half2 h01 = *reinterpret_cast<const __half2*>(&raw.x);
-    const __half2 h23 = *reinterpret_cast<const __half2*>(&raw.y);
-    float v[4] = {__low2float(h01), __high2float(h01), __low2float(h23), __high2float(h23)};
+  for (int blk0 = warp; blk0 < nblk; blk0 += 8 * p.NW) {
+    uint2 raw[8];
+    uint32_t sw[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if ((sw >> i) & 1u) v[i] = -v[i];
-    fwht128_warp(v, lane);
-    __half2 o01 = __floats2half2_rn(v[0] * kInvSqrt128, v[1] * kInvSqrt128);
-    __half2 o23 = __floats2half2_rn(v[2] * kInvSqrt128, v[3] * kInvSqrt128);
-    uint2 out;
-    out.x = *reinterpret_cast<uint32_t*>(&o01);
-    out.y = *reinterpret_cast<uint32_t*>(&o23);
-    *reinterpret_cast<uint2*>(xs + k0) = out;
+    for (int j = 0; j < 8; ++j) {
+      const int blk = blk0 + j * p.NW;
+      if (blk < nblk) {
+        raw[j] = *reinterpret_cast<const uint2*>(a.x + blk * kHadamard + 4 * lane);
+        sw[j] = a.sign_bits[blk * 4 + (lane >> 3)] >> (4 * (lane & 7));
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int blk = blk0 + j * p.NW;
+      if (blk >= nblk) break;
+      const __half2 h01 = *reinterpret_cast<const __half2*>(&raw[j].x);
+      const __half2 h23 = *reinterpret_cast<const __half2*>(&raw[j].y);
+      float v[4] = {__low2float(h01), __high2float(h01), __low2float(h23), __high2float(h23)};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if ((sw[j] >> i) & 1u) v[i] = -v[i];
+      fwht128_warp(v, lane);
+      __half2 o01 = __floats2half2_rn(v[0] * kInvSqrt128, v[1] * kInvSqrt128);
+      __half2 o23 = __floats2half2_rn(v[2] * kInvSqrt128, v[3] * kInvSqrt128);
+      uint2 out;
+      out.x = *reinterpret_cast<uint32_t*>(&o01);
+      out.y = *reinterpret_cast<uint32_t*>(&o23);
+      *reinterpret_cast<uint2*>(xs + blk * kHadamard + 4 * lane) = out;
+    }
   }
   named_barrier(1, ncons);
 
@@ -320,8 +388,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1) gemv1_kernel(const __grid_cons
   const int u = warp * p.UW + (lane % p.UW);
   const int row_sub = lane / p.UW;
   const bool active = row_sub < p.RS && u < p.U;
+  constexpr bool kIntPath = (B == 4 || B == 8);
   uint32_t xr[kXw];
-  float corr = 0.f, sx = 0.f;
+  float corr = 0.f, sx = 0.f, xinv = 1.f;
   if (active) {
     const uint4* xp = reinterpret_cast<const uint4*>(xs + (size_t)u * UT::kCodes);
 #pragma unroll
@@ -332,13 +401,53 @@ __global__ void __launch_bounds__(kMaxThreads, 1) gemv1_kernel(const __grid_cons
       xr[4 * i + 2] = v.z;
       xr[4 * i + 3] = v.w;
     }
+    if constexpr (kIntPath) {
+      // 16-bit integers with one power-of-two scale per unit: x_int = rne(x * 2^(13-E)),
+      // E the exponent of the unit's largest |x| (|x_int| < 2^14, exact for values
+      // within 2^4 of that maximum, else rounded at 2^(E-14)).
+      float m = 0.f;
 #pragma unroll
-    for (int i = 0; i < kXw; ++i) {
-      const __half2 h = *reinterpret_cast<const __half2*>(&xr[i]);
-      const float f0 = __low2float(h), f1 = __high2float(h);
-      sx += f0 + f1;
-      corr = fmaf(corr_weight<B>(2 * i), f0, corr);
-      corr = fmaf(corr_weight<B>(2 * i + 1), f1, corr);
+      for (int i = 0; i < kXw; ++i) {
+        const __half2 h = *reinterpret_cast<const __half2*>(&xr[i]);
+        m = fmaxf(m, fmaxf(fabsf(__low2float(h)), fabsf(__high2float(h))));
+      }
+      const int E = m > 0.f ? (int)((__float_as_uint(m) >> 23) & 0xFF) - 127 : 0;
+      const float up = __uint_as_float((uint32_t)(127 + 13 - E) << 23);
+      xinv = __uint_as_float((uint32_t)(127 - 13 + E) << 23);
+      uint32_t xi[kXw];
+      int isum = 0;
+#pragma unroll
+      for (int i = 0; i < kXw; ++i) {
+        const __half2 h = *reinterpret_cast<const __half2*>(&xr[i]);
+        const int v0 = __float2int_rn(__low2float(h) * up), v1 = __float2int_rn(__high2float(h) * up);
+        isum += v0 + v1;
+        const int s0 = int_slot<B>(2 * i), s1 = int_slot<B>(2 * i + 1);
+        reinterpret_cast<uint16_t*>(xi)[s0] = (uint16_t)v0;
+        reinterpret_cast<uint16_t*>(xi)[s1] = (uint16_t)v1;
+      }
+#pragma unroll
+      for (int i = 0; i < kXw; ++i) xr[i] = xi[i];
+      sx = (float)isum * xinv;
+    } else {
+#pragma unroll
+      for (int i = 0; i < kXw; ++i) {
+        const __half2 h = *reinterpret_cast<const __half2*>(&xr[i]);
+        const float f0 = __low2float(h), f1 = __high2float(h);
+        sx += f0 + f1;
+        corr = fmaf(corr_weight<B>(2 * i), f0, corr);
+        corr = fmaf(corr_weight<B>(2 * i + 1), f1, corr);
+      }
+    }
+  }
+  // Lanes on odd row slots read their unit's two 16-byte halves in the other
+  // order (bank-conflict-free unpadded rows); their x registers are swapped to match.
+  const int half_first = (UT::kBytes == 32 && p.swap_odd && (row_sub & 1)) ? 1 : 0;
+  if (half_first) {
+#pragma unroll
+    for (int i = 0; i < kXw / 2; ++i) {
+      const uint32_t t = xr[i];
+      xr[i] = xr[i + kXw / 2];
+      xr[i + kXw / 2] = t;
     }
   }
   const int g = (u * UT::kCodes) / kGroup;
@@ -353,22 +462,30 @@ __global__ void __launch_bounds__(kMaxThreads, 1) gemv1_kernel(const __grid_cons
     const __half* zsm = ssm + p.sz_halves;
     const int cr0 = t * Rc, cr = min(Rc, rows - cr0);
     const int aoff = (int)(((size_t)(n0 + cr0) * p.G) & 7);
+    // partial-sum rows of this chunk inside the window buffer
+    float* pchunk = part + (size_t)((t % p.chunks_per_window) * Rc) * p.U + u;
     if (active) {
-      for (int r = row_sub; r < cr; r += p.RS) {
-        const uint4* cp = reinterpret_cast<const uint4*>(st + (size_t)r * p.row_stride + u * UT::kBytes);
+      const uint8_t* cbase = st + u * UT::kBytes;
+      int r = row_sub;
+      // two rows per iteration: independent accumulator chains
+      for (; r + p.RS < cr; r += 2 * p.RS) {
+        const int r2 = r + p.RS;
+        uint32_t w[kWords], w2[kWords];
+        load_unit<kWords>(cbase + (size_t)r * p.row_stride, w, half_first);
+        load_unit<kWords>(cbase + (size_t)r2 * p.row_stride, w2, half_first);
+        const float d = unit_dot<B, kIntPath>(w, xr, corr, xinv);
+        const float d2 = unit_dot<B, kIntPath>(w2, xr, corr, xinv);
+        const float sc = __half2float(ssm[aoff + r * p.G + g]), zc = __half2float(zsm[aoff + r * p.G + g]);
+        const float sc2 = __half2float(ssm[aoff + r2 * p.G + g]), zc2 = __half2float(zsm[aoff + r2 * p.G + g]);
+        pchunk[(size_t)r * p.U] = sc * fmaf(-zc, sx, d);
+        pchunk[(size_t)r2 * p.U] = sc2 * fmaf(-zc2, sx, d2);
+      }
+      if (r < cr) {
         uint32_t w[kWords];
-#pragma unroll
-        for (int i = 0; i < kWords / 4; ++i) {
-          const uint4 v = cp[i];
-          w[4 * i] = v.x;
-          w[4 * i + 1] = v.y;
-          w[4 * i + 2] = v.z;
-          w[4 * i + 3] = v.w;
-        }
-        const float d = dot_unit(w, xr, int_<B>()) - corr;
-        const float sc = __half2float(ssm[aoff + r * p.G + g]);
-        const float zc = __half2float(zsm[aoff + r * p.G + g]);
-        part[((cr0 + r) % win_rows) * p.U + u] = sc * fmaf(-zc, sx, d);
+        load_unit<kWords>(cbase + (size_t)r * p.row_stride, w, half_first);
+        const float d = unit_dot<B, kIntPath>(w, xr, corr, xinv);
+        const float sc = __half2float(ssm[aoff + r * p.G + g]), zc = __half2float(zsm[aoff + r * p.G + g]);
+        pchunk[(size_t)r * p.U] = sc * fmaf(-zc, sx, d);
       }
     }
     __syncwarp();
@@ -394,28 +511,33 @@ int unit_bytes(int b) { return (b == 3 || b == 6) ? 48 : 32; }
 int unit_codes(int b) { return b == 3 ? 128 : (b == 8 ? 32 : 64); }
 
 // Worst bank-conflict degree of one 16-byte shared load by a warp whose lane l
-// reads row (l / UW) at unit (l % UW) with the given row stride.
-int conflict_degree(int UW, int RS, int ub, int stride) {
+// reads row (l / UW) at unit (l % UW) (two-piece units on odd rows swapped if asked).
+int conflict_degree(int UW, int RS, int ub, int stride, int swap_odd) {
   int worst = 1;
   for (int piece = 0; piece < ub / 16; ++piece)
     for (int ph = 0; ph < 4; ++ph) {
       int count[8] = {0};
       for (int l = ph * 8; l < ph * 8 + 8; ++l) {
-        if (l / UW >= RS) continue;
-        const long addr = (long)(l / UW) * stride + (long)(l % UW) * ub + 16 * piece;
+        const int row = l / UW;
+        if (row >= RS) continue;
+        const int pc = (ub == 32 && swap_odd && (row & 1)) ? (piece ^ 1) : piece;
+        const long addr = (long)row * stride + (long)(l % UW) * ub + 16 * pc;
         worst = std::max(worst, ++count[(addr / 16) % 8]);
       }
     }
   return worst;
 }
 
+int gemv1_ctas_per_sm(int b) { return b == 3 ? 1 : 2; }  // int3 lanes hold 64 registers of x
+
 bool make_plan(int b, int N, int K, Plan& p) {
   const int c = unit_codes(b), ub = unit_bytes(b);
+  const int max_warps = gemv1_ctas_per_sm(b) == 1 ? kMaxConsumerWarps : kMaxConsumerWarps2;
   p.U = K / c;
-  if (p.U < 1 || p.U > kMaxConsumerWarps * 32) return false;
+  if (p.U < 1 || p.U > max_warps * 32) return false;
   // Units per warp: most busy lanes, then most warps.
   double best = -1.0;
-  for (int UW = (p.U + kMaxConsumerWarps - 1) / kMaxConsumerWarps; UW <= 32 && UW <= p.U; ++UW) {
+  for (int UW = (p.U + max_warps - 1) / max_warps; UW <= 32 && UW <= p.U; ++UW) {
     const int RS = 32 / UW, NW = (p.U + UW - 1) / UW;
     const double eff = (double)RS * p.U / (NW * 32.0) + 1e-3 * NW;
     if (eff > best) {
@@ -427,16 +549,12 @@ bool make_plan(int b, int N, int K, Plan& p) {
   }
   p.row_bytes = K * b / 8;
   p.row_stride = p.row_bytes;
-  int bestc = 99;
-  for (int pad = 0; pad < 8; ++pad) {
-    const int cd = conflict_degree(p.UW, p.RS, ub, p.row_bytes + 16 * pad);
-    if (cd < bestc) {
-      bestc = cd;
-      p.row_stride = p.row_bytes + 16 * pad;
-    }
-  }
+  p.swap_odd = (ub == 32 && conflict_degree(p.UW, p.RS, ub, p.row_stride, 1) <
+                                conflict_degree(p.UW, p.RS, ub, p.row_stride, 0)) ? 1 : 0;
   p.G = K / kGroup;
-  p.grid = std::min(kSms, N);
+  p.ctas_per_sm = gemv1_ctas_per_sm(b);
+  const int smem_limit = p.ctas_per_sm == 1 ? kSmemLimit : kSmemLimit2;
+  p.grid = std::min(kSms * p.ctas_per_sm, N);
   p.rows_per_cta = (N + p.grid - 1) / p.grid;
   p.grid = (N + p.rows_per_cta - 1) / p.rows_per_cta;
   const int k = std::max(1, kChunkTarget / (p.RS * p.row_stride));
@@ -444,19 +562,19 @@ bool make_plan(int b, int N, int K, Plan& p) {
   const int nchunks = (p.rows_per_cta + p.rows_per_chunk - 1) / p.rows_per_chunk;
   p.sz_halves = ((p.rows_per_chunk * p.G + 8) + 7) & ~7;
   p.stage_bytes = (p.rows_per_chunk * p.row_stride + 4 * p.sz_halves + 127) & ~127;
-  const int max_win_chunks = std::max(1, kPartialBudget / (p.rows_per_chunk * p.U * 4));
+  const int max_win_chunks = std::max(1, kPartialBudget / p.ctas_per_sm / (p.rows_per_chunk * p.U * 4));
   p.chunks_per_window = std::min(max_win_chunks, nchunks);
   const int part_bytes = (p.chunks_per_window * p.rows_per_chunk * p.U * 4 + 127) & ~127;
   const int x_bytes = (K * 2 + 127) & ~127;
   const int fixed = x_bytes + part_bytes + 2 * kMaxStages * 8;
-  const int room = (kSmemLimit - fixed) / p.stage_bytes;
+  const int room = (smem_limit - fixed) / p.stage_bytes;
   p.stages = std::min(std::min(room, kMaxStages), nchunks);
   if (p.stages < 1) return false;
   p.off_x = p.stages * p.stage_bytes;
   p.off_part = p.off_x + x_bytes;
   p.off_bar = p.off_part + part_bytes;
   p.smem_bytes = p.off_bar + 2 * kMaxStages * 8;
-  return p.smem_bytes <= kSmemLimit;
+  return p.smem_bytes <= smem_limit;
 }
 
 template <int B>
@@ -466,12 +584,22 @@ qlin_status launch_gemv1(const Args& a, cudaStream_t s) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return record_cuda(e);
   if (dev >= 64 || !((configured >> dev) & 1ull)) {
-    e = cudaFuncSetAttribute(gemv1_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    e = cudaFuncSetAttribute(gemv1_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             gemv1_ctas_per_sm(B) == 1 ? kSmemLimit : kSmemLimit2);
     if (e != cudaSuccess) return record_cuda(e);
     if (dev < 64) configured |= 1ull << dev;
   }
-  gemv1_kernel<B><<<a.p.grid, (a.p.NW + 1) * 32, a.p.smem_bytes, s>>>(a);
-  return record_cuda(cudaGetLastError());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.p.grid);
+  cfg.blockDim = dim3((a.p.NW + 1) * 32);
+  cfg.dynamicSmemBytes = a.p.smem_bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = overlap_enabled() ? 1 : 0;
+  return record_cuda(cudaLaunchKernelEx(&cfg, gemv1_kernel<B>, a));
 }
 
 // ----------------------------------------------------- general fallback --

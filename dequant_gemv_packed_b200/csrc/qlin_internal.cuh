@@ -34,6 +34,7 @@ size_t code_bytes(const qlin_desc* d);
 size_t table_offset(const qlin_desc* d);
 PackedView make_view(const qlin_desc* d, const void* packed);
 qlin_status record_cuda(cudaError_t e);
+bool overlap_enabled();
 
 // Launchers (each returns QLIN_OK or QLIN_ERR_CUDA).
 qlin_status launch_pack(const PackedView& v, const uint8_t* codes, uint8_t* packed,

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "QLIN_OK", -1: "QLIN_ERR_INVALID_ARG", -2: "QLIN_ERR_UNSUPPOR
 EXPORTED = (
     "qlin_status_string", "qlin_last_cuda_error", "qlin_packed_bytes", "qlin_code_bytes", "qlin_pack",
     "qlin_unpack", "qlin_dequant", "qlin_rht", "qlin_gemv_workspace_bytes", "qlin_gemv",
-    "qlin_gemm_workspace_bytes", "qlin_gemm", "qlin_device_error", "qlin_gemm_noalloc",
+    "qlin_gemm_workspace_bytes", "qlin_gemm", "qlin_device_error", "qlin_gemm_noalloc", "qlin_set_overlap",
 )
 
 
@@ -76,6 +76,7 @@ def lib() -> ctypes.CDLL:
     vp, sz, i32, cp = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_char_p
     L.qlin_status_string.argtypes, L.qlin_status_string.restype = [ctypes.c_int], cp
     L.qlin_last_cuda_error.argtypes, L.qlin_last_cuda_error.restype = [], ctypes.c_int
+    L.qlin_set_overlap.argtypes, L.qlin_set_overlap.restype = [ctypes.c_int], ctypes.c_int
     L.qlin_packed_bytes.argtypes, L.qlin_packed_bytes.restype = [vp], sz
     L.qlin_code_bytes.argtypes, L.qlin_code_bytes.restype = [vp], sz
     L.qlin_pack.argtypes, L.qlin_pack.restype = [vp, vp, vp, vp], ctypes.c_int
@@ -126,6 +127,12 @@ def _alloc(shape, dtype, like: torch.Tensor) -> torch.Tensor:
 
 
 # ----------------------------------------------------------------- entry points
+
+def qlin_set_overlap(enable: bool) -> bool:
+    """Allow qlin_gemv to overlap the preceding kernel on its stream (see qlin.h);
+    returns the previous setting."""
+    return bool(lib().qlin_set_overlap(1 if enable else 0))
+
 
 def qlin_packed_bytes(desc: Desc) -> int:
     return int(lib().qlin_packed_bytes(desc.ref()))

@@ -110,6 +110,16 @@ const char* qlin_status_string(qlin_status status);
  * on the calling thread, 0 if none. */
 int qlin_last_cuda_error(void);
 
+/* Lets qlin_gemv (M = 1, uniform widths) overlap the kernel that precedes it on
+ * the stream (programmatic dependent launch): the call may start, and read its
+ * packed weight, scales, zeros and sign bits, before that kernel has finished;
+ * it waits for it before reading x or writing y.  This hides the launch and
+ * ramp of back-to-back calls, as in a decode loop over layers.  Enable it only
+ * if no kernel that writes the weight, scale, zero or sign buffers immediately
+ * precedes a call on the same stream.  Process-wide; default off.  Returns the
+ * previous setting. */
+int qlin_set_overlap(int enable);
+
 /* Bytes of the packed buffer for `desc` (codes, plus the block table for mixed
  * widths), a multiple of 16.  Returns 0 for an invalid descriptor. */
 size_t qlin_packed_bytes(const qlin_desc* desc);

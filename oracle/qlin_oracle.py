@@ -27,7 +27,7 @@ What it computes, in the plainest form that the pages support
 * ``linear64`` -- the fp64 matmul of the rotated activations with the fp64
   dequantised weight.
 
-Readings where the pages leave a step open (all listed in the design doc):
+Readings where the pages leave a step open (the library documents the same readings):
 
 * FWHT normalisation is 1/sqrt(128) (orthonormal): the pages call the transform
   orthogonal and function preserving.

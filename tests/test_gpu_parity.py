@@ -263,3 +263,37 @@ def test_zz_no_device_errors():
     """No bounded wait in any kernel gave up during the tests above."""
     torch.cuda.synchronize()
     assert Q.qlin_device_error() == 0
+
+
+def test_gemv_overlap_chain_matches_serial():
+    """With qlin_set_overlap(1), each call may start before the previous one ends;
+    a chain y_i = layer_i(y_{i-1}) must give the same bits as without overlap."""
+    K = 2560
+    layers = []
+    for i in range(6):
+        w = W.draw_weight(K, K, 4 if i % 2 == 0 else 8, seed=50 + i, device=DEV)
+        sb = W.draw_activation(1, K, seed=60 + i, device=DEV).sign_bits
+        d, packed = packed_on_device(w)
+        layers.append((d, packed, w.scales, w.zeros, sb))
+    x0 = W.draw_activation(1, K, seed=70, device=DEV).x
+
+    def chain(overlap):
+        prev = Q.qlin_set_overlap(overlap)
+        try:
+            x = x0
+            outs = []
+            for d, packed, s, z, sb in layers:
+                y = torch.empty(1, K, dtype=torch.float16, device=DEV)
+                Q.qlin_gemv(d, packed, s, z, sb, x, y)
+                # keep magnitudes bounded through the chain
+                x = y
+                outs.append(y)
+            torch.cuda.synchronize()
+            return [o.clone() for o in outs]
+        finally:
+            Q.qlin_set_overlap(prev)
+
+    serial, overlapped = chain(False), chain(True)
+    for a, b in zip(serial, overlapped):
+        assert torch.equal(a, b)
+    assert torch.isfinite(serial[-1].float()).all()
