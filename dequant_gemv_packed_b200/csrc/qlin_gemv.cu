@@ -10,34 +10,37 @@
 //
 // M = 1, uniform widths: gemv1_kernel.
 //   * One CTA per SM owns a contiguous range of weight rows.  A producer thread
-//     streams the rows (one bulk asynchronous copy per row, padded row stride
-//     in shared memory so that reads are bank-conflict free) and the group
-//     scales/zeros of each chunk of rows into a ring of shared-memory stages.
-//     All stages are issued before the prologue, so the whole HBM latency is
-//     overlapped with the rotation.
-//   * The consumer warps first rotate x (sign flip, 7 butterfly stages in
-//     registers and shuffles, x 1/sqrt(128), fp16 rounding) into shared memory.
-//   * Each consumer lane then owns one fixed "unit" of K (64 codes for int4 and
-//     int6, 128 for int3, 32 for int8) and keeps its slice of rotated x in
-//     registers for the whole kernel, walking down the rows of each chunk.
-//   * 4- and 8-bit codes: the lane converts its rotated x to 16-bit integers
-//     with one power-of-two scale per unit (exact for values within 2^4 of the
-//     unit's largest magnitude, else rounded at 2^-14 of it) and takes
-//     sum_k q_k x_k exactly in int32 with dp2a (two 16x8-bit products per
-//     instruction); nibbles are spread to byte lanes with one mask each.
+//     streams the rows (one bulk asynchronous copy per chunk of rows, laid out
+//     in shared memory exactly as in global memory) and the group scales/zeros
+//     of each chunk into a ring of shared-memory stages; when the CTA's whole
+//     share fits (the common decode shapes), every chunk has its own stage and
+//     all copies are in flight before the first x value is read.
+//   * The consumer warps rotate x (sign flip, 7 butterfly stages in registers
+//     and shuffles, x 1/sqrt(128), fp16 rounding) and, in the same pass, put
+//     each "unit" of K (64 codes; 32 for int8) into the form its decoder
+//     reads, with the unit's scalars (below).
+//   * Each consumer lane then owns one fixed unit, keeps that unit's x in
+//     registers for the whole kernel, and walks down the rows of each chunk;
+//     the UW lanes that share a row (UW a power of two) add their per-unit
+//     results with shuffles, and rows are summed over warps in a fixed order
+//     (deterministic results).
+//   * 4- and 8-bit codes: x becomes 16-bit integers with one power-of-two scale
+//     per unit (exact for values within 2^4 of the unit's largest magnitude,
+//     else rounded at 2^-14 of it) and sum_k q_k x_k is taken exactly in int32
+//     with dp2a (two 16x8-bit products per instruction); nibbles are spread to
+//     byte lanes with one mask each.
 //   * 3- and 6-bit codes are turned into fp16 without conversions: masking a
 //     code into the mantissa of the fp16 constant 1024 (0x6400) gives exactly
 //     1024 + c*q, where c is a power of two fixed by the code's bit position;
 //     one lop3 produces two such values.  They are multiplied with x in fp16 x
 //     fp16 -> fp32 fused multiply-adds, one accumulator per position scale c,
-//     and the constant part 1024*sum(x/c) is removed afterwards with a
-//     correction computed once per lane from its x registers.
-//   * Per (row, unit) the lane stores s*(sum q x - z*sum x) to shared memory;
-//     rows are summed over units in a fixed order (deterministic results).
+//     and the constant part 1024*sum(x/c) is removed with the unit's
+//     correction.
 //   * With qlin_set_overlap(1) the kernel is launched as a programmatic
 //     dependent: it lets the next kernel start launching at once, streams its
 //     weight before waiting on the previous kernel, and waits only before it
-//     reads x (so back-to-back calls overlap their ramp and drain).
+//     reads x; two CTAs fit on an SM, so the next call's weight stream runs
+//     under this call's arithmetic.
 // Other cases (M > 1, mixed widths): the activation rotation runs as its own
 // kernel into the workspace, then gemv_simple_kernel.
 #include <algorithm>
@@ -52,40 +55,41 @@ __device__ unsigned int g_gemv_error;  // nonzero: a bounded wait gave up
 namespace {
 
 constexpr uint32_t kMagic = 0x64006400u;  // fp16 1024.0 in both halves
-constexpr int kMaxConsumerWarps = 16;
+// Two CTAs fit on one SM (registers and shared memory), so that with
+// programmatic dependent launch the next call's CTA is resident, and streams
+// its weight, while this call's CTA finishes.
+constexpr int kMaxConsumerWarps = 10;
 constexpr int kMaxThreads = (kMaxConsumerWarps + 1) * 32;
-// Two CTAs per SM: at most 10 consumer warps each, so registers stay <= 93.
-constexpr int kMaxConsumerWarps2 = 10;
-constexpr int kMaxThreads2 = (kMaxConsumerWarps2 + 1) * 32;
-constexpr int kSmemLimit = 227 * 1024;      // one CTA per SM
-constexpr int kSmemLimit2 = 113 * 1024;     // two CTAs per SM
-constexpr int kChunkTarget = 24 * 1024;
-constexpr int kPartialBudget = 48 * 1024;
+constexpr int kSmemLimit = 113 * 1024;
+constexpr int kMinSmem = 80 * 1024;
+constexpr int kChunkTarget = 16 * 1024;
+constexpr int kInflightBytes = 64 * 1024;
+constexpr int kPartialBudget = 24 * 1024;
 constexpr int kMaxStages = 16;
 constexpr int kSms = 148;
 
 template <int N> struct int_ {};
 
+// A unit is the run of codes one lane multiplies with its x registers.
 template <int B> struct UnitT;
-template <> struct UnitT<3> { static constexpr int kBytes = 48, kCodes = 128; };
+template <> struct UnitT<3> { static constexpr int kBytes = 24, kCodes = 64; };
 template <> struct UnitT<4> { static constexpr int kBytes = 32, kCodes = 64; };
 template <> struct UnitT<6> { static constexpr int kBytes = 48, kCodes = 64; };
 template <> struct UnitT<8> { static constexpr int kBytes = 32, kCodes = 32; };
 
 struct Plan {
   int U;               // units per row
-  int UW, RS, NW;      // units per warp, row slots per warp, consumer warps
-  int rows_per_cta, grid;
-  int row_bytes, row_stride;  // row_stride == row_bytes: a chunk is one contiguous copy
-  int swap_odd;        // 32-byte units: lanes on odd row slots read their two halves swapped
-  int ctas_per_sm;
-  int rows_per_chunk;  // R_c, a multiple of RS
+  int UW, RS, NW;      // units per warp (a power of two), row slots per warp (32 / UW), consumer warps
+  int rows_per_cta, grid;  // rows_per_cta: the most rows one CTA owns
+  int row_bytes;       // rows are contiguous in shared memory as in global memory
+  int swap_bit;        // 32-byte units: lanes with this lane-index bit set read their halves swapped (-1: none)
+  int rows_per_chunk;  // R_c, a multiple of the rows one consumer iteration covers
+  int inflight;        // chunks of one CTA in flight at once
   int stages;
   int chunks_per_window;
   int G;               // groups per row
   int sz_halves;       // halves per stage for each of s and z
-  int stage_bytes;
-  int off_x, off_part, off_bar;
+  int off_sz, off_x, off_unit, off_part, off_bar;
   int smem_bytes;
 };
 
@@ -97,12 +101,11 @@ struct Args {
   const __half* x;
   __half* y;
   int N, K;
+  int weights_first;  // dependent launch: stream the weight before waiting for x
   Plan p;
 };
 
 // ---------------------------------------------------------------- decoders --
-// Each returns sum_k (1024/c_k + q_k) * x_k over the unit, where c_k is the
-// position scale of code k; the lane subtracts corr = sum_k 1024/c_k * x_k.
 
 // Integer decoders (4- and 8-bit codes): dp2a multiplies two signed 16-bit
 // activations by two unsigned 8-bit codes and adds to an int32, exactly.
@@ -120,45 +123,40 @@ __device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int c) {
 }
 
 // int4: word i holds codes 8i..8i+7.  x pairs: (x0,x2) (x4,x6) (x1,x3) (x5,x7).
+// The odd codes are used in place (16 q in the high nibble of each byte), so
+// their sums carry a factor 16 that is shifted out at the end (exactly: the sum
+// is a multiple of 16).
 __device__ __forceinline__ int dot_unit_int(const uint32_t (&w)[8], const uint32_t (&x)[32], int_<4>) {
-  int a0 = 0, a1 = 0;
+  int lo0 = 0, lo1 = 0, hi0 = 0, hi1 = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t lo = w[i] & 0x0F0F0F0Fu;         // q0 q2 q4 q6
-    const uint32_t hi = (w[i] >> 4) & 0x0F0F0F0Fu;  // q1 q3 q5 q7
-    int& A = (i & 1) ? a1 : a0;
-    A = dp2a_lo(x[4 * i], lo, A);
-    A = dp2a_hi(x[4 * i + 1], lo, A);
-    A = dp2a_lo(x[4 * i + 2], hi, A);
-    A = dp2a_hi(x[4 * i + 3], hi, A);
+    const uint32_t lo = w[i] & 0x0F0F0F0Fu;  // q0 q2 q4 q6
+    const uint32_t hi = w[i] & 0xF0F0F0F0u;  // 16 q1, 16 q3, 16 q5, 16 q7
+    int& L = (i & 1) ? lo1 : lo0;
+    int& H = (i & 1) ? hi1 : hi0;
+    L = dp2a_lo(x[4 * i], lo, L);
+    L = dp2a_hi(x[4 * i + 1], lo, L);
+    H = dp2a_lo(x[4 * i + 2], hi, H);
+    H = dp2a_hi(x[4 * i + 3], hi, H);
   }
-  return a0 + a1;
+  return (lo0 + lo1) + ((hi0 + hi1) >> 4);
 }
 
 // int8: word i holds codes 4i..4i+3.  x pairs: (x0,x1) (x2,x3).
 __device__ __forceinline__ int dot_unit_int(const uint32_t (&w)[8], const uint32_t (&x)[16], int_<8>) {
-  int a0 = 0, a1 = 0;
+  int acc[4] = {0, 0, 0, 0};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    int& A = (i & 1) ? a1 : a0;
+    int& A = acc[i & 3];
     A = dp2a_lo(x[2 * i], w[i], A);
     A = dp2a_hi(x[2 * i + 1], w[i], A);
   }
-  return a0 + a1;
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
-// Position of code c (0-based within the unit) in the lane's int16 x layout.
-template <int B>
-__device__ __forceinline__ int int_slot(int c) {
-  if (B == 8) return c;  // natural order
-  // int4: word i = c/8, code j = c%8 -> pair order (0,2) (4,6) (1,3) (5,7)
-  const int i = c >> 3, j = c & 7;
-  const int pair = ((j & 1) << 1) | (j >> 2);  // j=0,2 ->0; 4,6 ->1; 1,3 ->2; 5,7 ->3
-  return 8 * i + 2 * pair + ((j >> 1) & 1);
-}
-
-// 48 bits of a 48-byte unit starting at bit 48*p: A = bits [0, 32), B = bits [32, 48) (+ junk above).
-__device__ __forceinline__ void piece48(const uint32_t (&w)[12], int p, uint32_t& A, uint32_t& B) {
+// 48 bits of a unit starting at bit 48*p: A = bits [0, 32), B = bits [32, 48) (+ junk above).
+template <int kWords>
+__device__ __forceinline__ void piece48(const uint32_t (&w)[kWords], int p, uint32_t& A, uint32_t& B) {
   const int m = p >> 1;
   if ((p & 1) == 0) {
     A = w[3 * m];
@@ -169,8 +167,10 @@ __device__ __forceinline__ void piece48(const uint32_t (&w)[12], int p, uint32_t
   }
 }
 
-__device__ __forceinline__ float dot_unit(const uint32_t (&w)[12], const uint32_t (&x)[32],
-                                          int_<6>) {
+// The fp16 decoders (3- and 6-bit codes) return sum_k (1024/c_k + q_k) * x_k
+// over the unit, where c_k is the position scale of code k; the caller
+// subtracts corr = sum_k 1024/c_k * x_k.
+__device__ __forceinline__ float dot_unit(const uint32_t (&w)[12], const uint32_t (&x)[32], int_<6>) {
   float a1a = 0.f, a1b = 0.f, a4a = 0.f, a4b = 0.f;
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
@@ -196,11 +196,11 @@ __device__ __forceinline__ float dot_unit(const uint32_t (&w)[12], const uint32_
   return (a1a + a1b) + 0.25f * (a4a + a4b);
 }
 
-__device__ __forceinline__ float dot_unit(const uint32_t (&w)[12], const uint32_t (&x)[64],
-                                          int_<3>) {
+// int3: a 64-code unit is four 48-bit pieces of 16 codes.
+__device__ __forceinline__ float dot_unit(const uint32_t (&w)[6], const uint32_t (&x)[32], int_<3>) {
   float a1 = 0.f, a2 = 0.f, a8 = 0.f, a16 = 0.f, a64 = 0.f, a128 = 0.f;
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
+  for (int p = 0; p < 4; ++p) {
     uint32_t A, B;
     piece48(w, p, A, B);
     const uint32_t u0 = A << 1;
@@ -214,7 +214,7 @@ __device__ __forceinline__ float dot_unit(const uint32_t (&w)[12], const uint32_
     const uint32_t R = ((A >> 9) & 0x3Fu) | (B << 15);
     const uint32_t T6 = (R & 0x00070007u) | kMagic;   // (q3, q11)
     const uint32_t T7 = (R & 0x00380038u) | kMagic;   // (8 q4, 8 q12)
-    const uint32_t* xp = x + 8 * p;  // xp[i] = (x_{2i}, x_{2i+1}) of this pair of pieces
+    const uint32_t* xp = x + 8 * p;  // xp[i] = (x_{2i}, x_{2i+1}) of this piece
     a2 = fma_f16f32(lo16(T0), lo16(xp[0]), a2);
     a1 = fma_f16f32(hi16(T0), hi16(xp[2]), a1);
     a16 = fma_f16f32(lo16(T1), hi16(xp[0]), a16);
@@ -235,311 +235,483 @@ __device__ __forceinline__ float dot_unit(const uint32_t (&w)[12], const uint32_
   return a1 + 0.5f * a2 + 0.125f * a8 + 0.0625f * a16 + 0.015625f * a64 + 0.0078125f * a128;
 }
 
-// 1024 / c for code position i of a unit (see the decoders above).
+// 1024 / c for code position i of a unit (see the fp16 decoders above): a
+// power of two whose exponent, for i mod 8, is a nibble of a constant (no
+// branches: lanes ask for different positions).
 template <int B>
 __device__ __forceinline__ float corr_weight(int i) {
-  if (B == 8) return 1024.f;
-  if (B == 4) return (i & 1) ? 64.f : 1024.f;
-  if (B == 6) {
-    const int r = i & 7;
-    return (r == 3 || r == 4 || r == 5 || r == 7) ? 256.f : 1024.f;
-  }
-  // B == 3, period 16
-  const int r = i & 15;
-  switch (r & 7) {
-    case 0: return 512.f;
-    case 1: return 64.f;
-    case 2: return 8.f;
-    case 3: return 1024.f;
-    case 4: return 128.f;
-    case 5: return 1024.f;
-    case 6: return 128.f;
-    default: return 16.f;
-  }
+  // int6: 1024 except 256 at positions 3, 4, 5, 7; int3: 512 64 8 1024 128 1024 128 16
+  constexpr uint32_t kExp = B == 6 ? 0x8A888AAAu : 0x47A7A369u;
+  const uint32_t e = (kExp >> (4 * (i & 7))) & 0xFu;
+  return __uint_as_float((127u + e) << 23);
 }
 
 __device__ __forceinline__ void gemv_fail(unsigned code) { atomicOr(&g_gemv_error, code); }
 
 // sum_k q_k x_k over one unit: exact integer dot (scaled back) or the fp16
-// mantissa-code path minus its constant part.
+// mantissa-code path minus its constant part.  `c` is the unit's scale
+// 2^(E-13) (integer path) or its correction (fp16 path).
 template <int B, bool kInt, int kWords, int kXw>
-__device__ __forceinline__ float unit_dot(const uint32_t (&w)[kWords], const uint32_t (&x)[kXw], float corr,
-                                          float xinv) {
+__device__ __forceinline__ float unit_dot(const uint32_t (&w)[kWords], const uint32_t (&x)[kXw], float c) {
   if constexpr (kInt) {
-    return (float)dot_unit_int(w, x, int_<B>()) * xinv;
+    return (float)dot_unit_int(w, x, int_<B>()) * c;
   } else {
-    return dot_unit(w, x, int_<B>()) - corr;
+    return dot_unit(w, x, int_<B>()) - c;
   }
 }
 
+// One unit of codes from shared memory (16-byte pieces, or 8-byte pieces for
+// 24-byte units); `half_first` swaps the two 16-byte halves of a 32-byte unit.
 template <int kWords>
-__device__ __forceinline__ void load_unit(const uint8_t* src, uint32_t (&w)[kWords], int half_first = 0) {
-  const uint4* cp = reinterpret_cast<const uint4*>(src);
+__device__ __forceinline__ void load_unit(const uint8_t* src, uint32_t (&w)[kWords], int half_first) {
+  if constexpr (kWords % 4 == 0) {
+    const uint4* cp = reinterpret_cast<const uint4*>(src);
 #pragma unroll
-  for (int i = 0; i < kWords / 4; ++i) {
-    const uint4 v = cp[kWords == 8 ? (i ^ half_first) : i];
-    w[4 * i] = v.x;
-    w[4 * i + 1] = v.y;
-    w[4 * i + 2] = v.z;
-    w[4 * i + 3] = v.w;
+    for (int i = 0; i < kWords / 4; ++i) {
+      const uint4 v = cp[kWords == 8 ? (i ^ half_first) : i];
+      w[4 * i] = v.x;
+      w[4 * i + 1] = v.y;
+      w[4 * i + 2] = v.z;
+      w[4 * i + 3] = v.w;
+    }
+  } else {
+    const uint2* cp = reinterpret_cast<const uint2*>(src);
+#pragma unroll
+    for (int i = 0; i < kWords / 2; ++i) {
+      const uint2 v = cp[i];
+      w[2 * i] = v.x;
+      w[2 * i + 1] = v.y;
+    }
+  }
+}
+
+// Rows per consumer iteration: four for int4; two for int3 and int6 (registers) and
+// int8 (long rows: smaller chunks keep more ring stages).
+template <int B> struct RowsPerIter { static constexpr int value = B == 4 ? 4 : 2; };
+
+// The UW lanes of a row group hold per-unit partials v[k] of the R rows
+// rb + k RS (k < R).  A reduce-scatter butterfly leaves the full sum of row
+// k = (lane & (min(R, UW) - 1)) in each lane (log2(R) exchange steps that halve
+// the values a lane carries, then a plain butterfly over the remaining lane
+// bits); the lanes of the group's first min(R, UW) holding distinct rows store
+// them.  Every lane of the warp executes it.
+template <int UW, int R>
+__device__ __forceinline__ void reduce_store_rows(float (&v)[R], int lane, float* pchunk, int r0, int RS, int cr,
+                                                  int NW) {
+  if constexpr (UW == 1) {
+#pragma unroll
+    for (int k = 0; k < R; ++k)
+      if (r0 + k * RS < cr) pchunk[(r0 + k * RS) * NW] = v[k];
+  } else {
+    constexpr int kSplit = UW < R ? UW : R;  // lanes that end up with distinct rows
+    float c[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) c[k] = v[k];
+    int n = R;  // values still carried
+#pragma unroll
+    for (int o = kSplit / 2; o >= 1; o /= 2) {
+      // keep the upper or lower half of the carried values, add the partner's copy
+      const bool upper = (lane & o) != 0;
+      n /= 2;
+#pragma unroll
+      for (int k = 0; k < R / 2; ++k) {
+        if (k < n) {
+          const float keep = upper ? c[k + n] : c[k];
+          const float send = upper ? c[k] : c[k + n];
+          c[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+    }
+    // c[0 .. n) now hold rows (lane & (kSplit-1)) * n + j; finish over the other lane bits
+#pragma unroll
+    for (int o = kSplit; o < UW; o *= 2)
+#pragma unroll
+      for (int k = 0; k < R; ++k)
+        if (k < n) c[k] += __shfl_xor_sync(0xffffffffu, c[k], o);
+    if ((lane & (UW - 1)) < kSplit) {
+      const int kb = (lane & (kSplit - 1)) * n;
+#pragma unroll
+      for (int j = 0; j < R; ++j)
+        if (j < n && r0 + (kb + j) * RS < cr) pchunk[(r0 + (kb + j) * RS) * NW] = c[j];
+    }
   }
 }
 
 // ------------------------------------------------------------------ kernel --
 
+// Maximum (of non-negative values) and sum over the lanes of this lane's group
+// (grp in [0, kGroups)): one warp-wide redux per group.
+template <int kGroups>
+__device__ __forceinline__ uint32_t group_max(uint32_t m, int grp) {
+  uint32_t r = 0;
+#pragma unroll
+  for (int q = 0; q < kGroups; ++q) {
+    const uint32_t mq = __reduce_max_sync(0xffffffffu, grp == q ? m : 0u);
+    if (grp == q) r = mq;
+  }
+  return r;
+}
+template <int kGroups>
+__device__ __forceinline__ int group_add(int v, int grp) {
+  int r = 0;
+#pragma unroll
+  for (int q = 0; q < kGroups; ++q) {
+    const int sq = __reduce_add_sync(0xffffffffu, grp == q ? v : 0);
+    if (grp == q) r = sq;
+  }
+  return r;
+}
+
+// (H[r][c], H[r][c+1]) of the Sylvester matrix of order 16 as two fp16 (+-1).
+__device__ __forceinline__ uint32_t h16_pair(int r, int c) {
+  const uint32_t lo = (__popc(r & c) & 1) ? 0xBC00u : 0x3C00u;
+  const uint32_t hi = (__popc(r & (c + 1)) & 1) ? 0xBC00u : 0x3C00u;
+  return lo | (hi << 16);
+}
+
+// Position in dp2a order of code c of a 64-code int4 unit (pairs (0,2) (4,6)
+// (1,3) (5,7) of each word of 8 codes; see dot_unit_int).
+__device__ __forceinline__ int int4_slot(int c) {
+  const int j = c & 7;
+  return 8 * (c >> 3) + 2 * (((j & 1) << 1) | (j >> 2)) + ((j >> 1) & 1);
+}
+
+// Sign flip, block-128 FWHT, x 1/sqrt(128) and fp16 rounding of one block,
+// then the unit preparation described at the top of the file.
+// The order-128 Sylvester matrix is H16 (x) H8 (element e = i + 16 j: bits
+// 0-3 and 4-6 of e), so with X[i][j] = d_e x_e the rotation is H16 X H8: one
+// m16n8k16 tensor-core product (A = H16, B = X) and three butterfly stages
+// along j.  Lane (g, t) = (lane / 4, lane % 4) supplies X[2t, 2t+1][g] and
+// X[2t+8, 2t+9][g] (x at 16g + 2t and 16g + 2t + 8: b0 and b1, signs in sw)
+// and ends with elements g + 32t + {0, 16, 8, 24}.
 template <int B>
-__global__ void __launch_bounds__(B == 3 ? kMaxThreads : kMaxThreads2, B == 3 ? 1 : 2)
-    gemv1_kernel(const __grid_constant__ Args a) {
+__device__ __forceinline__ void rotate_prepare(uint32_t b0, uint32_t b1, uint32_t sw, int blk, bool store,
+                                               const uint32_t (&h)[4], uint32_t* xs, float2* ust, int lane) {
   using UT = UnitT<B>;
+  constexpr int kXw = UT::kCodes / 2;
+  const int g = lane >> 2, t = lane & 3;
+  b0 ^= ((sw & 1u) << 15) | ((sw & 2u) << 30);
+  b1 ^= (((sw >> 8) & 1u) << 15) | (((sw >> 8) & 2u) << 30);
+  float c0, c1, c2, c3;
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+      : "=f"(c0), "=f"(c1), "=f"(c2), "=f"(c3)
+      : "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3]), "r"(b0), "r"(b1), "f"(0.f));
+  // columns 2t, 2t+1 (stride 1 in j), then partners t^1 and t^2 (strides 2, 4)
+  float v[4] = {c0 + c1, c0 - c1, c2 + c3, c2 - c3};
+#pragma unroll
+  for (int o = 1; o <= 2; o <<= 1) {
+    const bool up = (t & o) != 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float q = __shfl_xor_sync(0xffffffffu, v[i], o);
+      v[i] = up ? q - v[i] : v[i] + q;
+    }
+  }
+  constexpr int kOff[4] = {0, 16, 8, 24};  // element of v[i]: g + 32 t + kOff[i]
+  __half hv[4];
+  float f[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    hv[i] = __float2half_rn(v[i] * kInvSqrt128);
+    f[i] = __half2float(hv[i]);
+  }
+  // units: 64 codes = elements [0, 64) or [64, 128) of the block (t < 2 or t >= 2);
+  // 32 codes (int8) = the 32 elements of one t
+  constexpr int kGroups = UT::kCodes == 64 ? 2 : 4;
+  const int grp = UT::kCodes == 64 ? (t >> 1) : t;
+  const int u = blk * (kHadamard / UT::kCodes) + grp;
+  const bool leader = g == 0 && (UT::kCodes == 32 || (t & 1) == 0);
+  uint16_t* xu = reinterpret_cast<uint16_t*>(xs + (size_t)u * kXw);
+  if constexpr (B == 4 || B == 8) {
+    // x_int = rne(x * 2^(13-E)), E the exponent of the unit's largest |x|:
+    // |x_int| < 2^14, exact for values within 2^4 of that maximum.
+    const uint32_t m = group_max<kGroups>(
+        __float_as_uint(fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])))), grp);
+    const int E = m ? (int)((m >> 23) & 0xFF) - 127 : 0;
+    const float up = __uint_as_float((uint32_t)(127 + 13 - E) << 23);
+    const float xinv = __uint_as_float((uint32_t)(127 - 13 + E) << 23);
+    int vi[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) vi[i] = __float2int_rn(f[i] * up);
+    const int isum = group_add<kGroups>((vi[0] + vi[1]) + (vi[2] + vi[3]), grp);
+    if (store) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = (B == 4) ? g + 32 * (t & 1) + kOff[i] : g + kOff[i];  // position in the unit
+        xu[B == 4 ? int4_slot(c) : c] = (uint16_t)vi[i];
+      }
+      if (leader) ust[u] = make_float2(xinv, (float)isum * xinv);
+    }
+  } else {
+    float corr = 0.f, sx = (f[0] + f[1]) + (f[2] + f[3]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) corr = fmaf(corr_weight<B>(g + 32 * (t & 1) + kOff[i]), f[i], corr);
+#pragma unroll
+    for (int o = 1; o <= 16; o <<= 1) {
+      if (o == 2) continue;  // lane bit 1 selects the unit
+      corr += __shfl_xor_sync(0xffffffffu, corr, o);
+      sx += __shfl_xor_sync(0xffffffffu, sx, o);
+    }
+    if (store) {
+      __half* xh = reinterpret_cast<__half*>(xs) + (size_t)blk * kHadamard + g + 32 * t;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xh[kOff[i]] = hv[i];
+      if (leader) ust[u] = make_float2(corr, sx);
+    }
+  }
+}
+
+template <int B, int UW>
+__global__ void __launch_bounds__(kMaxThreads, 2) gemv1_kernel(const __grid_constant__ Args a) {
+  using UT = UnitT<B>;
+  constexpr int R = RowsPerIter<B>::value;
   constexpr int kWords = UT::kBytes / 4;
-  constexpr int kXw = UT::kCodes / 2;  // half2 registers of x per lane
+  constexpr int kXw = UT::kCodes / 2;  // 32-bit registers of x per lane
+  constexpr bool kIntPath = (B == 4 || B == 8);
   extern __shared__ __align__(128) uint8_t smem[];
   const Plan& p = a.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ncons = p.NW * 32;
-  const int n0 = blockIdx.x * p.rows_per_cta;
-  const int rows = min(p.rows_per_cta, a.N - n0);
+  // CTA i owns rows [i N / grid, (i + 1) N / grid): every SM gets work.
+  const int n0 = (int)(((long long)blockIdx.x * a.N) / gridDim.x);
+  const int rows = (int)(((long long)(blockIdx.x + 1) * a.N) / gridDim.x) - n0;
   if (rows <= 0) return;
   const int Rc = p.rows_per_chunk;
   const int nchunks = (rows + Rc - 1) / Rc;
+  const size_t stage_bytes = (size_t)Rc * p.row_bytes;
+  uint8_t* codes_ring = smem;  // stage s holds rows [0, Rc) of its chunk at s * Rc * row_bytes
+  __half* s_ring = reinterpret_cast<__half*>(smem + p.off_sz);
+  __half* z_ring = s_ring + p.stages * p.sz_halves;
+  uint32_t* xs = reinterpret_cast<uint32_t*>(smem + p.off_x);
+  float2* ust = reinterpret_cast<float2*>(smem + p.off_unit);
+  float* part = reinterpret_cast<float*>(smem + p.off_part);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   uint64_t* empty = full + kMaxStages;
-  __half* xs = reinterpret_cast<__half*>(smem + p.off_x);
-  float* part = reinterpret_cast<float*>(smem + p.off_part);
+  uint64_t* x_issued = empty + kMaxStages;
 
   if (tid == ncons) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], p.NW);
     }
+    mbar_init(x_issued, p.NW);
     mbar_fence_init();
   }
   __syncthreads();
   // Programmatic dependent launch: the next kernel on the stream may start
-  // launching now; this kernel's own weight stream does not depend on the
+  // launching now; this kernel's weight stream does not depend on the
   // previous kernel, x and y do (grid_dependency_wait below).
   if (tid == 0) grid_launch_dependents();
 
   if (warp == p.NW) {
     // ------------------------------------------------------- producer ----
     if (lane != 0) return;
+    // Stand-alone launches let the x loads go first (the weight stream would
+    // otherwise queue ahead of them); dependent launches stream at once.
+    if (!a.weights_first && !mbar_wait(x_issued, 0, &g_gemv_error)) gemv_fail(4u);
+    const size_t total_h = (size_t)a.N * p.G;
+    int s = 0, sd = 0;
+    uint32_t ph = 0, phd = 0;
     for (int t = 0; t < nchunks; ++t) {
-      const int s = t % p.stages;
-      if (t >= p.stages && !mbar_wait(&empty[s], ((t / p.stages) - 1) & 1, &g_gemv_error)) gemv_fail(1u);
-      uint8_t* st = smem + (size_t)s * p.stage_bytes;
-      __half* ssm = reinterpret_cast<__half*>(st + (size_t)Rc * p.row_stride);
-      __half* zsm = ssm + p.sz_halves;
+      if (t >= p.stages && !mbar_wait(&empty[s], ph ^ 1u, &g_gemv_error)) gemv_fail(1u);
+      // Pace the stream: at most p.inflight chunks of this CTA in flight, so
+      // that the first chunks land early instead of all together.
+      if (t >= p.inflight) {
+        if (!mbar_wait(&full[sd], phd, &g_gemv_error)) gemv_fail(8u);
+        if (++sd == p.stages) {
+          sd = 0;
+          phd ^= 1u;
+        }
+      }
+      uint8_t* dst = codes_ring + (size_t)s * stage_bytes;
+      __half* ssm = s_ring + (size_t)s * p.sz_halves;
+      __half* zsm = z_ring + (size_t)s * p.sz_halves;
       const int cr0 = t * Rc, cr = min(Rc, rows - cr0);
       const size_t h0 = (size_t)(n0 + cr0) * p.G, h1 = h0 + (size_t)cr * p.G;
-      const size_t al = h0 & ~(size_t)7, bl = h1 & ~(size_t)7;
-      for (size_t h = (bl > h0 ? bl : h0); h < h1; ++h) {  // unaligned tail: plain copies
-        ssm[h - al] = a.scales[h];
-        zsm[h - al] = a.zeros[h];
+      const size_t al = h0 & ~(size_t)7;
+      size_t bh = (h1 + 7) & ~(size_t)7;  // whole 16-byte pieces, reading a little past the chunk
+      if (bh > total_h) {                 // ... except at the end of the arrays: plain copies
+        bh = h1 & ~(size_t)7;
+        for (size_t h = (bh > h0 ? bh : h0); h < h1; ++h) {
+          ssm[h - al] = a.scales[h];
+          zsm[h - al] = a.zeros[h];
+        }
       }
-      const uint32_t szb = bl > al ? (uint32_t)(bl - al) * 2u : 0u;
+      const uint32_t szb = bh > al ? (uint32_t)(bh - al) * 2u : 0u;
       mbar_arrive_expect_tx(&full[s], (uint32_t)cr * p.row_bytes + 2u * szb);
-      bulk_g2s(st, a.codes + (size_t)(n0 + cr0) * p.row_bytes, (uint32_t)cr * p.row_bytes, &full[s]);
+      bulk_g2s(dst, a.codes + (size_t)(n0 + cr0) * p.row_bytes, (uint32_t)cr * p.row_bytes, &full[s]);
       if (szb) {
         bulk_g2s(ssm, a.scales + al, szb, &full[s]);
         bulk_g2s(zsm, a.zeros + al, szb, &full[s]);
+      }
+      if (++s == p.stages) {
+        s = 0;
+        ph ^= 1u;
       }
     }
     return;
   }
 
   // --------------------------------------------------------- prologue ----
-  // Rotate x into shared memory: warp per block of 128, lane holds 4 values.
-  // All of a warp's x loads are issued before any is used (one memory latency).
+  // Rotate x and prepare each unit in shared memory in the form the decoders
+  // read (rotate_prepare): warp per block of 128, two blocks per pass.  All of
+  // a warp's x loads are issued before any is used (one memory latency).
   grid_dependency_wait();
   const int nblk = a.K / kHadamard;
-  for (int blk0 = warp; blk0 < nblk; blk0 += 8 * p.NW) {
-    uint2 raw[8];
-    uint32_t sw[8];
+  constexpr int kBatch = 8;
+  if (warp >= nblk && lane == 0) mbar_arrive(x_issued);  // a warp with no block has nothing to load
+  {
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t h[4] = {h16_pair(g, 2 * t), h16_pair(g + 8, 2 * t), h16_pair(g, 2 * t + 8),
+                           h16_pair(g + 8, 2 * t + 8)};
+    const int xo = 16 * g + 2 * t;                 // x offset of this lane's b0 (b1: + 8)
+    const int so = (g >> 1), sb = 16 * (g & 1) + 2 * t;  // its sign word and bit
+    for (int blk0 = warp; blk0 < nblk; blk0 += kBatch * p.NW) {
+      uint32_t xb0[kBatch], xb1[kBatch], sw[kBatch];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int blk = blk0 + j * p.NW;
-      if (blk < nblk) {
-        raw[j] = *reinterpret_cast<const uint2*>(a.x + blk * kHadamard + 4 * lane);
-        sw[j] = a.sign_bits[blk * 4 + (lane >> 3)] >> (4 * (lane & 7));
+      for (int j = 0; j < kBatch; ++j) {
+        const int blk = min(blk0 + j * p.NW, nblk - 1);
+        const __half* xp = a.x + blk * kHadamard + xo;
+        xb0[j] = *reinterpret_cast<const uint32_t*>(xp);
+        xb1[j] = *reinterpret_cast<const uint32_t*>(xp + 8);
+        sw[j] = a.sign_bits[blk * 4 + so] >> sb;
       }
-    }
+      if (blk0 == warp) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(x_issued);
+      }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int blk = blk0 + j * p.NW;
-      if (blk >= nblk) break;
-      const __half2 h01 = *reinterpret_cast<const __half2*>(&raw[j].x);
-      const __half2 h23 = *reinterpret_cast<const __half2*>(&raw[j].y);
-      float v[4] = {__low2float(h01), __high2float(h01), __low2float(h23), __high2float(h23)};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if ((sw[j] >> i) & 1u) v[i] = -v[i];
-      fwht128_warp(v, lane);
-      __half2 o01 = __floats2half2_rn(v[0] * kInvSqrt128, v[1] * kInvSqrt128);
-      __half2 o23 = __floats2half2_rn(v[2] * kInvSqrt128, v[3] * kInvSqrt128);
-      uint2 out;
-      out.x = *reinterpret_cast<uint32_t*>(&o01);
-      out.y = *reinterpret_cast<uint32_t*>(&o23);
-      *reinterpret_cast<uint2*>(xs + blk * kHadamard + 4 * lane) = out;
+      for (int j = 0; j < kBatch; j += 2) {
+        const int b0 = blk0 + j * p.NW, b1 = b0 + p.NW;
+        if (b0 >= nblk) break;  // warp-uniform
+        rotate_prepare<B>(xb0[j], xb1[j], sw[j], b0, true, h, xs, ust, lane);
+        rotate_prepare<B>(xb0[j + 1], xb1[j + 1], sw[j + 1], min(b1, nblk - 1), b1 < nblk, h, xs, ust, lane);
+      }
     }
   }
   named_barrier(1, ncons);
 
-  // Fixed unit of this lane, its x slice in registers, and its corrections.
-  const int u = warp * p.UW + (lane % p.UW);
-  const int row_sub = lane / p.UW;
-  const bool active = row_sub < p.RS && u < p.U;
-  constexpr bool kIntPath = (B == 4 || B == 8);
+  // Fixed unit of this lane: x slice in registers, unit scalars.
+  const int u = warp * UW + (lane & (UW - 1));
+  const int row_sub = lane / UW;
+  const bool unit_ok = u < p.U;
+  const int uc = unit_ok ? u : p.U - 1;  // lanes past the last unit read a valid unit, contribute 0
+  const int half_first = (UT::kBytes == 32 && p.swap_bit >= 0) ? ((lane >> p.swap_bit) & 1) : 0;
   uint32_t xr[kXw];
-  float corr = 0.f, sx = 0.f, xinv = 1.f;
-  if (active) {
-    const uint4* xp = reinterpret_cast<const uint4*>(xs + (size_t)u * UT::kCodes);
+  {
+    const uint4* xp = reinterpret_cast<const uint4*>(xs + (size_t)uc * kXw);
 #pragma unroll
     for (int i = 0; i < kXw / 4; ++i) {
-      const uint4 v = xp[i];
+      const uint4 v = xp[i ^ (half_first * (kXw / 8))];
       xr[4 * i] = v.x;
       xr[4 * i + 1] = v.y;
       xr[4 * i + 2] = v.z;
       xr[4 * i + 3] = v.w;
     }
-    if constexpr (kIntPath) {
-      // 16-bit integers with one power-of-two scale per unit: x_int = rne(x * 2^(13-E)),
-      // E the exponent of the unit's largest |x| (|x_int| < 2^14, exact for values
-      // within 2^4 of that maximum, else rounded at 2^(E-14)).
-      float m = 0.f;
-#pragma unroll
-      for (int i = 0; i < kXw; ++i) {
-        const __half2 h = *reinterpret_cast<const __half2*>(&xr[i]);
-        m = fmaxf(m, fmaxf(fabsf(__low2float(h)), fabsf(__high2float(h))));
-      }
-      const int E = m > 0.f ? (int)((__float_as_uint(m) >> 23) & 0xFF) - 127 : 0;
-      const float up = __uint_as_float((uint32_t)(127 + 13 - E) << 23);
-      xinv = __uint_as_float((uint32_t)(127 - 13 + E) << 23);
-      uint32_t xi[kXw];
-      int isum = 0;
-#pragma unroll
-      for (int i = 0; i < kXw; ++i) {
-        const __half2 h = *reinterpret_cast<const __half2*>(&xr[i]);
-        const int v0 = __float2int_rn(__low2float(h) * up), v1 = __float2int_rn(__high2float(h) * up);
-        isum += v0 + v1;
-        const int s0 = int_slot<B>(2 * i), s1 = int_slot<B>(2 * i + 1);
-        reinterpret_cast<uint16_t*>(xi)[s0] = (uint16_t)v0;
-        reinterpret_cast<uint16_t*>(xi)[s1] = (uint16_t)v1;
-      }
-#pragma unroll
-      for (int i = 0; i < kXw; ++i) xr[i] = xi[i];
-      sx = (float)isum * xinv;
-    } else {
-#pragma unroll
-      for (int i = 0; i < kXw; ++i) {
-        const __half2 h = *reinterpret_cast<const __half2*>(&xr[i]);
-        const float f0 = __low2float(h), f1 = __high2float(h);
-        sx += f0 + f1;
-        corr = fmaf(corr_weight<B>(2 * i), f0, corr);
-        corr = fmaf(corr_weight<B>(2 * i + 1), f1, corr);
-      }
-    }
   }
-  // Lanes on odd row slots read their unit's two 16-byte halves in the other
-  // order (bank-conflict-free unpadded rows); their x registers are swapped to match.
-  const int half_first = (UT::kBytes == 32 && p.swap_odd && (row_sub & 1)) ? 1 : 0;
-  if (half_first) {
-#pragma unroll
-    for (int i = 0; i < kXw / 2; ++i) {
-      const uint32_t t = xr[i];
-      xr[i] = xr[i + kXw / 2];
-      xr[i + kXw / 2] = t;
-    }
-  }
-  const int g = (u * UT::kCodes) / kGroup;
-  const int win_rows = p.chunks_per_window * Rc;
+  const float2 us = ust[uc];
+  const float uscale = us.x, sx = us.y;
+  const int g = (uc * UT::kCodes) / kGroup;
+  const uint8_t* lane_codes = codes_ring + uc * UT::kBytes;
+  const int G = p.G, RS = p.RS, NW = p.NW, row_bytes = p.row_bytes;
+  const bool ring = p.stages < nchunks;  // stages are reused: release each one when done
 
   // -------------------------------------------------------- main loop ----
+  int s = 0, wt = 0, wr0 = 0, cr0 = 0;
+  uint32_t ph = 0;
+  int aoff = (int)(((size_t)n0 * G) & 7);  // offset of the chunk's first scale in its 16-byte-aligned copy
+  const int aoff_step = (Rc * G) & 7;
   for (int t = 0; t < nchunks; ++t) {
-    const int s = t % p.stages;
-    if (!mbar_wait(&full[s], (t / p.stages) & 1, &g_gemv_error)) gemv_fail(2u);
-    const uint8_t* st = smem + (size_t)s * p.stage_bytes;
-    const __half* ssm = reinterpret_cast<const __half*>(st + (size_t)Rc * p.row_stride);
-    const __half* zsm = ssm + p.sz_halves;
-    const int cr0 = t * Rc, cr = min(Rc, rows - cr0);
-    const int aoff = (int)(((size_t)(n0 + cr0) * p.G) & 7);
-    // partial-sum rows of this chunk inside the window buffer
-    float* pchunk = part + (size_t)((t % p.chunks_per_window) * Rc) * p.U + u;
-    if (active) {
-      const uint8_t* cbase = st + u * UT::kBytes;
-      int r = row_sub;
-      // two rows per iteration: independent accumulator chains
-      for (; r + p.RS < cr; r += 2 * p.RS) {
-        const int r2 = r + p.RS;
-        uint32_t w[kWords], w2[kWords];
-        load_unit<kWords>(cbase + (size_t)r * p.row_stride, w, half_first);
-        load_unit<kWords>(cbase + (size_t)r2 * p.row_stride, w2, half_first);
-        const float d = unit_dot<B, kIntPath>(w, xr, corr, xinv);
-        const float d2 = unit_dot<B, kIntPath>(w2, xr, corr, xinv);
-        const float sc = __half2float(ssm[aoff + r * p.G + g]), zc = __half2float(zsm[aoff + r * p.G + g]);
-        const float sc2 = __half2float(ssm[aoff + r2 * p.G + g]), zc2 = __half2float(zsm[aoff + r2 * p.G + g]);
-        pchunk[(size_t)r * p.U] = sc * fmaf(-zc, sx, d);
-        pchunk[(size_t)r2 * p.U] = sc2 * fmaf(-zc2, sx, d2);
+    if (!mbar_wait_poll(&full[s], ph, &g_gemv_error)) gemv_fail(2u);
+    const int cr = min(Rc, rows - cr0);
+    const uint8_t* cbase = lane_codes + (size_t)s * stage_bytes;
+    const __half* sp = s_ring + (size_t)s * p.sz_halves + aoff + g;
+    const __half* zp = z_ring + (size_t)s * p.sz_halves + aoff + g;
+    float* pchunk = part + (size_t)(wt * Rc) * NW + warp;
+    // R rows per iteration (independent accumulator chains).  Every lane runs
+    // every iteration (the row sums are warp shuffles); lanes whose row is at
+    // or past `cr` read the chunk's last row instead and store nothing.
+    for (int rb = 0; rb < cr; rb += R * RS) {
+      const int r0 = rb + row_sub;
+      uint32_t w[R][kWords];
+      float sc[R], zc[R], v[R];
+#pragma unroll
+      for (int k = 0; k < R; ++k) {
+        const int rl = min(r0 + k * RS, cr - 1);
+        load_unit<kWords>(cbase + rl * row_bytes, w[k], half_first);
+        sc[k] = __half2float(sp[rl * G]);
+        zc[k] = __half2float(zp[rl * G]);
       }
-      if (r < cr) {
-        uint32_t w[kWords];
-        load_unit<kWords>(cbase + (size_t)r * p.row_stride, w, half_first);
-        const float d = unit_dot<B, kIntPath>(w, xr, corr, xinv);
-        const float sc = __half2float(ssm[aoff + r * p.G + g]), zc = __half2float(zsm[aoff + r * p.G + g]);
-        pchunk[(size_t)r * p.U] = sc * fmaf(-zc, sx, d);
+#pragma unroll
+      for (int k = 0; k < R; ++k) {
+        const float d = unit_dot<B, kIntPath>(w[k], xr, uscale);
+        v[k] = unit_ok ? sc[k] * fmaf(-zc[k], sx, d) : 0.f;
       }
+      reduce_store_rows<UW, R>(v, lane, pchunk, r0, RS, cr, NW);
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-    if ((t + 1) % p.chunks_per_window == 0 || t + 1 == nchunks) {
+    if (ring) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    if (++s == p.stages) {
+      s = 0;
+      ph ^= 1u;
+    }
+    aoff = (aoff + aoff_step) & 7;
+    cr0 += Rc;
+    if (++wt == p.chunks_per_window || t + 1 == nchunks) {
       named_barrier(1, ncons);
-      const int wr0 = (t / p.chunks_per_window) * win_rows;
-      const int wrows = min(win_rows, rows - wr0);
+      const int wrows = min(wt * Rc, rows - wr0);
       for (int rr = tid; rr < wrows; rr += ncons) {
-        const float* pr = part + (size_t)rr * p.U;
+        const float* pr = part + (size_t)rr * NW;
         float acc = 0.f;
-        for (int uu = 0; uu < p.U; ++uu) acc += pr[uu];
+        for (int ww = 0; ww < NW; ++ww) acc += pr[ww];
         a.y[n0 + wr0 + rr] = __float2half_rn(acc);
       }
       named_barrier(1, ncons);
+      wr0 += wt * Rc;
+      wt = 0;
     }
   }
 }
 
 // ------------------------------------------------------------- host plan --
 
-int unit_bytes(int b) { return (b == 3 || b == 6) ? 48 : 32; }
-int unit_codes(int b) { return b == 3 ? 128 : (b == 8 ? 32 : 64); }
+int unit_bytes(int b) { return b == 3 ? 24 : (b == 6 ? 48 : 32); }
+int unit_codes(int b) { return b == 8 ? 32 : 64; }
 
-// Worst bank-conflict degree of one 16-byte shared load by a warp whose lane l
-// reads row (l / UW) at unit (l % UW) (two-piece units on odd rows swapped if asked).
-int conflict_degree(int UW, int RS, int ub, int stride, int swap_odd) {
+// Worst bank-conflict degree of one shared load (16-byte pieces, 8-byte pieces
+// for 24-byte units) by a warp whose lane l reads row (l / UW) at unit (l % UW);
+// 32-byte units of lanes with bit `swap_bit` set are read second half first.
+int conflict_degree(int UW, int ub, int stride, int swap_bit) {
+  const int aw = ub % 16 ? 8 : 16, per_phase = 128 / aw, groups = 128 / aw;
   int worst = 1;
-  for (int piece = 0; piece < ub / 16; ++piece)
-    for (int ph = 0; ph < 4; ++ph) {
-      int count[8] = {0};
-      for (int l = ph * 8; l < ph * 8 + 8; ++l) {
+  for (int piece = 0; piece < ub / aw; ++piece)
+    for (int ph = 0; ph < 32 / per_phase; ++ph) {
+      int count[16] = {0};
+      for (int l = ph * per_phase; l < (ph + 1) * per_phase; ++l) {
         const int row = l / UW;
-        if (row >= RS) continue;
-        const int pc = (ub == 32 && swap_odd && (row & 1)) ? (piece ^ 1) : piece;
-        const long addr = (long)row * stride + (long)(l % UW) * ub + 16 * pc;
-        worst = std::max(worst, ++count[(addr / 16) % 8]);
+        const int pc = (ub == 32 && swap_bit >= 0 && ((l >> swap_bit) & 1)) ? (piece ^ 1) : piece;
+        const long addr = (long)row * stride + (long)(l % UW) * ub + (long)aw * pc;
+        worst = std::max(worst, ++count[(addr / aw) % groups]);
       }
     }
   return worst;
 }
 
-int gemv1_ctas_per_sm(int b) { return b == 3 ? 1 : 2; }  // int3 lanes hold 64 registers of x
-
 bool make_plan(int b, int N, int K, Plan& p) {
   const int c = unit_codes(b), ub = unit_bytes(b);
-  const int max_warps = gemv1_ctas_per_sm(b) == 1 ? kMaxConsumerWarps : kMaxConsumerWarps2;
+  if (K % c) return false;
   p.U = K / c;
-  if (p.U < 1 || p.U > max_warps * 32) return false;
-  // Units per warp: most busy lanes, then most warps.
+  if (p.U < 1 || p.U > kMaxConsumerWarps * 32) return false;
+  // Units per warp (a power of two): most busy lanes, then most warps.
+  // Row slots beyond the rows a CTA owns would idle.
+  const int rows_est = (N + std::min(kSms, N) - 1) / std::min(kSms, N);
   double best = -1.0;
-  for (int UW = (p.U + max_warps - 1) / max_warps; UW <= 32 && UW <= p.U; ++UW) {
+  for (int UW = 1; UW <= 32; UW *= 2) {
     const int RS = 32 / UW, NW = (p.U + UW - 1) / UW;
-    const double eff = (double)RS * p.U / (NW * 32.0) + 1e-3 * NW;
+    if (NW > kMaxConsumerWarps) continue;
+    const double eff = (double)std::min(RS, rows_est) * p.U / (NW * 32.0) + 1e-3 * NW;
     if (eff > best) {
       best = eff;
       p.UW = UW;
@@ -547,45 +719,71 @@ bool make_plan(int b, int N, int K, Plan& p) {
       p.NW = NW;
     }
   }
+  if (best < 0) return false;
   p.row_bytes = K * b / 8;
-  p.row_stride = p.row_bytes;
-  p.swap_odd = (ub == 32 && conflict_degree(p.UW, p.RS, ub, p.row_stride, 1) <
-                                conflict_degree(p.UW, p.RS, ub, p.row_stride, 0)) ? 1 : 0;
+  p.swap_bit = -1;
+  if (ub == 32) {
+    int worst = conflict_degree(p.UW, ub, p.row_bytes, -1);
+    for (int bit = 0; bit < 5; ++bit) {
+      const int d = conflict_degree(p.UW, ub, p.row_bytes, bit);
+      if (d < worst) {
+        worst = d;
+        p.swap_bit = bit;
+      }
+    }
+  }
   p.G = K / kGroup;
-  p.ctas_per_sm = gemv1_ctas_per_sm(b);
-  const int smem_limit = p.ctas_per_sm == 1 ? kSmemLimit : kSmemLimit2;
-  p.grid = std::min(kSms * p.ctas_per_sm, N);
-  p.rows_per_cta = (N + p.grid - 1) / p.grid;
-  p.grid = (N + p.rows_per_cta - 1) / p.rows_per_cta;
-  const int k = std::max(1, kChunkTarget / (p.RS * p.row_stride));
-  p.rows_per_chunk = std::min(p.RS * k, ((p.rows_per_cta + p.RS - 1) / p.RS) * p.RS);
+  p.grid = std::min(kSms, N);
+  p.rows_per_cta = (N + p.grid - 1) / p.grid;  // the most rows a CTA owns
+  const int step = (b == 4 ? 4 : 2) * p.RS;  // rows per consumer iteration (RowsPerIter)
+  const int k = std::max(1, (kChunkTarget + step * p.row_bytes / 2) / (step * p.row_bytes));
+  p.rows_per_chunk = std::min(step * k, ((p.rows_per_cta + step - 1) / step) * step);
   const int nchunks = (p.rows_per_cta + p.rows_per_chunk - 1) / p.rows_per_chunk;
-  p.sz_halves = ((p.rows_per_chunk * p.G + 8) + 7) & ~7;
-  p.stage_bytes = (p.rows_per_chunk * p.row_stride + 4 * p.sz_halves + 127) & ~127;
-  const int max_win_chunks = std::max(1, kPartialBudget / p.ctas_per_sm / (p.rows_per_chunk * p.U * 4));
-  p.chunks_per_window = std::min(max_win_chunks, nchunks);
-  const int part_bytes = (p.chunks_per_window * p.rows_per_chunk * p.U * 4 + 127) & ~127;
+  p.sz_halves = (p.rows_per_chunk * p.G + 16 + 7) & ~7;
   const int x_bytes = (K * 2 + 127) & ~127;
-  const int fixed = x_bytes + part_bytes + 2 * kMaxStages * 8;
-  const int room = (smem_limit - fixed) / p.stage_bytes;
-  p.stages = std::min(std::min(room, kMaxStages), nchunks);
-  if (p.stages < 1) return false;
-  p.off_x = p.stages * p.stage_bytes;
-  p.off_part = p.off_x + x_bytes;
-  p.off_bar = p.off_part + part_bytes;
-  p.smem_bytes = p.off_bar + 2 * kMaxStages * 8;
-  return p.smem_bytes <= smem_limit;
+  const int unit_scalars = (p.U * 8 + 127) & ~127;
+  const int sz_stage = 4 * p.sz_halves;
+  const auto part_bytes = [&](int cpw) { return (cpw * p.rows_per_chunk * p.NW * 4 + 127) & ~127; };
+  const int bars = (2 * kMaxStages + 1) * 8;
+  // The whole share in shared memory at once (each chunk its own stage)?
+  const int codes_all = (p.rows_per_cta * p.row_bytes + 127) & ~127;
+  const int single = codes_all + ((nchunks * sz_stage + 127) & ~127) + x_bytes + unit_scalars +
+                     part_bytes(nchunks) + bars;
+  if (nchunks <= kMaxStages && single <= kSmemLimit) {
+    p.stages = nchunks;
+    p.chunks_per_window = nchunks;
+    p.off_sz = codes_all;
+  } else {
+    const int max_win_chunks = std::max(1, kPartialBudget / (p.rows_per_chunk * p.NW * 4));
+    p.chunks_per_window = std::min(max_win_chunks, nchunks);
+    const int fixed = x_bytes + unit_scalars + part_bytes(p.chunks_per_window) + bars;
+    const int stage_cost = p.rows_per_chunk * p.row_bytes + sz_stage;
+    p.stages = std::min(std::min((kSmemLimit - fixed - 256) / stage_cost, kMaxStages), nchunks);
+    if (p.stages < 1) return false;
+    p.off_sz = (p.stages * p.rows_per_chunk * p.row_bytes + 127) & ~127;
+  }
+  // About 64 KB of one CTA's stream in flight (148 CTAs: ~9.5 MB, enough to cover
+  // the memory latency at full bandwidth).
+  p.inflight = std::max(1, std::min(p.stages, (kInflightBytes + p.rows_per_chunk * p.row_bytes - 1) /
+                                                  (p.rows_per_chunk * p.row_bytes)));
+  p.off_x = (p.off_sz + p.stages * sz_stage + 127) & ~127;
+  p.off_unit = p.off_x + x_bytes;
+  p.off_part = p.off_unit + unit_scalars;
+  p.off_bar = p.off_part + part_bytes(p.chunks_per_window);
+  // At least kMinSmem per CTA, so that no more than two calls' CTAs share an SM
+  // (the one running and the next, prefetching), whatever their shapes.
+  p.smem_bytes = std::max(p.off_bar + bars, kMinSmem);
+  return p.off_bar + bars <= kSmemLimit;
 }
 
-template <int B>
-qlin_status launch_gemv1(const Args& a, cudaStream_t s) {
+template <int B, int UW>
+qlin_status launch_gemv1_uw(const Args& a, cudaStream_t s) {
   static unsigned long long configured = 0;  // one bit per device (the attribute is per device)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return record_cuda(e);
   if (dev >= 64 || !((configured >> dev) & 1ull)) {
-    e = cudaFuncSetAttribute(gemv1_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             gemv1_ctas_per_sm(B) == 1 ? kSmemLimit : kSmemLimit2);
+    e = cudaFuncSetAttribute(gemv1_kernel<B, UW>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     if (e != cudaSuccess) return record_cuda(e);
     if (dev < 64) configured |= 1ull << dev;
   }
@@ -599,7 +797,19 @@ qlin_status launch_gemv1(const Args& a, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = overlap_enabled() ? 1 : 0;
-  return record_cuda(cudaLaunchKernelEx(&cfg, gemv1_kernel<B>, a));
+  return record_cuda(cudaLaunchKernelEx(&cfg, gemv1_kernel<B, UW>, a));
+}
+
+template <int B>
+qlin_status launch_gemv1(const Args& a, cudaStream_t s) {
+  switch (a.p.UW) {
+    case 1: return launch_gemv1_uw<B, 1>(a, s);
+    case 2: return launch_gemv1_uw<B, 2>(a, s);
+    case 4: return launch_gemv1_uw<B, 4>(a, s);
+    case 8: return launch_gemv1_uw<B, 8>(a, s);
+    case 16: return launch_gemv1_uw<B, 16>(a, s);
+    default: return launch_gemv1_uw<B, 32>(a, s);
+  }
 }
 
 // ----------------------------------------------------- general fallback --
@@ -666,6 +876,7 @@ qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half*
       a.y = y;
       a.N = v.N;
       a.K = v.K;
+      a.weights_first = overlap_enabled() ? 1 : 0;
       switch (v.bits) {
         case 3: return launch_gemv1<3>(a, s);
         case 4: return launch_gemv1<4>(a, s);

@@ -77,6 +77,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   return false;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait for a phase that has usually completed already: a few cheap
+// non-blocking tests first (no suspension when the data is there), then the
+// bounded blocking wait.
+__device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, const volatile unsigned* abort_word) {
+#pragma unroll 1
+  for (int i = 0; i < 4; ++i)
+    if (mbar_test_wait(bar, parity)) return true;
+  return mbar_wait(bar, parity, abort_word);
+}
+
 // Bulk copy of `bytes` (multiple of 16; both addresses 16-byte aligned) from
 // global to this CTA's shared memory, completing on `bar` (tx bytes).
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

@@ -163,6 +163,16 @@ def test_gemv_ragged(bits, N, K, M):
     _gemv_case(w, a, what=f"b{bits} N{N} K{K} M{M}")
 
 
+@pytest.mark.parametrize("bits", [3, 4, 6, 8])
+@pytest.mark.parametrize("N,K", [(77, 384), (149, 128), (333, 1280), (64, 9728), (1337, 2560), (4440, 4096)])
+def test_gemv_m1_shapes(bits, N, K):
+    """M = 1 across row counts that leave ragged chunks and idle lanes, shares
+    that fit shared memory whole and ones that cycle the stage ring."""
+    w = _rand_weight(N, K, bits, seed=3 * N + bits)
+    a = W.draw_activation(1, K, seed=N + 1).to(DEV)
+    _gemv_case(w, a, what=f"b{bits} N{N} K{K} M1")
+
+
 def test_gemv_mixed():
     bb = [6, 8, 4, 3, 8]
     w = _rand_weight(64 * len(bb), 1280, 0, seed=5, block_bits=bb)
