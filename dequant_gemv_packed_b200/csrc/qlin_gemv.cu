@@ -785,6 +785,12 @@ qlin_status launch_gemv1_uw(const Args& a, cudaStream_t s) {
   if (dev >= 64 || !((configured >> dev) & 1ull)) {
     e = cudaFuncSetAttribute(gemv1_kernel<B, UW>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     if (e != cudaSuccess) return record_cuda(e);
+    // Every instance asks for the largest shared-memory carveout, so that
+    // consecutive calls of different shapes find the SM configured alike and
+    // the next call's CTA fits beside the running one.
+    e = cudaFuncSetAttribute(gemv1_kernel<B, UW>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return record_cuda(e);
     if (dev < 64) configured |= 1ull << dev;
   }
   cudaLaunchConfig_t cfg = {};
