@@ -81,7 +81,7 @@ def kernel_source_hash() -> str:
 def ncu_traffic(workload: str, kernel_hash: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel sources; else None."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    p = os.path.join(ROOT, "profiles", "traffic.txt")  # JSON text
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(workload)
@@ -147,15 +147,21 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def dist_setup():
+def dist_setup(backend: str | None = None):
+    """One process per GPU under torchrun (RANK/LOCAL_RANK/WORLD_SIZE/MASTER_* from
+    the environment): NCCL on GPUs; `backend="gloo"` runs the same plumbing on CPU."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if world > 1:
         import datetime
         import torch.distributed as dist
         local = int(os.environ.get("LOCAL_RANK", "0"))
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        backend = backend or "nccl"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
         return dist, dist.get_rank(), world, local
     return None, 0, 1, 0
 
@@ -166,11 +172,19 @@ def barrier(dist):
 
 
 def max_over_ranks(dist, v: float) -> float:
+    """The largest of the ranks' values (every rank gets it)."""
     if dist is None:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_gbs(bytes_per_step: int, steps: int, world: int, ms_max: float) -> float:
+    """Weak scaling: every rank runs `steps` calls of `bytes_per_step`; the job's
+    throughput is all ranks' bytes over the slowest rank's time."""
+    return world * bytes_per_step * steps / (ms_max * 1e-3) / 1e9
 
 
 # ------------------------------------------------------------------- workloads
@@ -432,7 +446,7 @@ def run_ours(args):
     ms, clocks = time_steps(case, args.steps, args.warmup, dist, stream)
     ms_step = ms / args.steps
     peaks = measured_peaks()
-    value = world * case.bytes * args.steps / (ms * 1e-3) / 1e9
+    value = whole_job_gbs(case.bytes, args.steps, world, ms)
     per_gpu_gbs = case.bytes / (ms_step * 1e-3) / 1e9
     khash = kernel_source_hash()
     if case.kind == "gemm":

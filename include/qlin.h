@@ -167,9 +167,18 @@ size_t qlin_gemv_workspace_bytes(const qlin_desc* desc, int32_t M);
 
 /* Decode-regime quantised linear layer, 1 <= M <= 16:
  *   y[m][n] = fp16_rn( sum_k rht(x)[m][k] * w[n][k] ), fp32 accumulation,
- * with rht(x) rounded to fp16 as qlin_rht does.  Weights are dequantised in
- * registers and never written to memory; the per-group scale and zero may be
- * applied to the group's partial sum, sum_k s(q - z)x = s(sum qx - z sum x).
+ * with rht(x) rounded once to fp16.  Weights are dequantised in registers and
+ * never written to memory; the per-group scale and zero may be applied to the
+ * group's partial sum, sum_k s(q - z)x = s(sum qx - z sum x).
+ * The M = 1 kernel (uniform widths) rotates x itself, evaluating the block
+ * transform as H16 (x) H8 with one tensor-core product per block (fp32
+ * accumulation; a rotated value can differ from qlin_rht's by one fp16 ulp
+ * where the exact value lies near a rounding boundary), and for 4- and 8-bit
+ * codes multiplies the rotated x as 16-bit integers with one power-of-two
+ * scale per 64 (int8: 32) consecutive values: exact for values within a
+ * factor 16 of the largest magnitude of their run, others rounded at 2^-14 of
+ * it.  These readings are judged by the output tolerance, like the factored
+ * scale.
  *   x : device fp16 [M][K] (not rotated);  y : device fp16 [M][N];
  *   workspace : device buffer of workspace_bytes >= qlin_gemv_workspace_bytes(M, K)
  *               bytes (may be NULL when that is 0); overwritten.
