@@ -1,22 +1,29 @@
 // qlin_gemm: prefill-regime quantised linear layer on the 5th-generation tensor
-// cores (tcgen05, accumulators in tensor memory).
+// cores (tcgen05, operands and accumulators in tensor memory).
 //
 // Y = rht(X) . dequant(W)^T.  The activations are rotated into the workspace
 // by the stand-alone rotation kernel; the weight is dequantised exactly as
-// qlin_dequant does (fp32 subtract and multiply, one rounding to fp16) into
-// shared memory, inside the main loop, and never reaches global memory
+// qlin_dequant does (fp32 subtract and multiply, one rounding to fp16) straight
+// into tensor memory, inside the main loop, and never reaches global memory
 // ("24B0978-Week01-Track2_20-Submission01", "How these techniques accelerate
 // inference on CUDA").
 //
 // Tiling (one CTA per SM, persistent over output tiles):
 //   MMA  D[128 weight rows][BN activation rows] += A[128][64] . B[BN][64]^T
-//   A = dequantised weight rows, K-major, 128-byte swizzle, written by 8
-//       dequantisation warps straight from the packed codes in global memory;
-//   B = rotated activations, K-major, 128-byte swizzle, loaded by TMA;
-//   D = fp32 in tensor memory, two accumulators (2 x 256 columns) so the
-//       epilogue of one tile overlaps the main loop of the next.
+//   A = dequantised weight rows in tensor memory (row m in lane m, two fp16
+//       along K per 32-bit column), one 32-column slot per pipeline stage,
+//       written by 8 dequantisation warps with tcgen05.st;
+//   B = rotated activations in shared memory, K-major, 128-byte swizzle,
+//       loaded by TMA;
+//   D = fp32 in tensor memory, columns [0, BN).
 // Warp roles: 0 TMA producer, 1 MMA issuer (one thread) and TMEM owner,
 // 4..7 epilogue (TMEM lane quarters 0..3), 8..15 dequantisation.
+// Dequantisation warp 8 + j owns TMEM lane quarter q = j % 4 (weight rows
+// 32q .. 32q+31 of the tile, one per thread) and half h = j / 4 of every
+// 64-code stage.  Each thread copies its own row's two 32-code pieces of every
+// 128-code group kRing groups ahead (cp.async into a private ring slot), so the
+// dequantisation warps never wait for one another; results go to tensor memory,
+// which the MMA reads without a proxy fence.
 // The weight tile is the MMA's M side because dequantisation costs ALU work
 // per weight element per activation tile: with 256 activation rows per tile
 // each weight element is dequantised once per 256 rows of X.
@@ -35,24 +42,21 @@ __device__ unsigned int g_gemm_error;
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kBK = 64;        // k per stage: 64 fp16 = one 128-byte swizzle row
+constexpr int kBK = 64;        // k per stage: 64 fp16 = one 128-byte swizzle row of B
 constexpr int kBMw = 128;      // weight rows per tile (MMA M)
 constexpr int kBNmax = 256;    // activation rows per tile (MMA N)
-constexpr int kAStage = kBMw * kBK * 2;     // 16 KB
 constexpr int kBStage = kBNmax * kBK * 2;   // 32 KB
 constexpr int kThreads = 512;
 constexpr int kDeqWarp0 = 8, kDeqWarps = 8;
+constexpr int kDeqThreads = kDeqWarps * 32;
 constexpr int kEpiWarp0 = 4;
 constexpr int kTmemCols = 512;
-// Codes of one 128-code group of the whole 128-row weight tile (two MMA
-// stages), copied cooperatively and coalesced by the dequantisation threads
-// into a ring of kCodeRing slots: row r at r * 128 bytes, its 16-byte piece c
-// at slot (c ^ (r & 7)) (bank-conflict-free reads of the row slices).
-constexpr int kDeqThreads = kDeqWarps * 32;
-constexpr int kCodeRing = 2;
-constexpr int kCodeSlotBytes = kBMw * 128;
-constexpr int kSmemBytes = kStages * (kAStage + kBStage) + kCodeRing * kCodeSlotBytes + 1024 /*barriers*/ +
-                           1024 /*align*/;
+constexpr int kAccCol = 0;     // accumulator: columns [0, BN)
+constexpr int kACol = 256;     // A of stage s: columns [kACol + 32 s, kACol + 32 s + 32)
+constexpr int kRing = 4;       // 128-code groups in flight per dequantisation thread
+constexpr int kSlot = 80;      // bytes per thread per group: pieces at 0 and 32 (16-byte stride 5: no bank conflicts)
+constexpr int kRingBytes = kRing * kDeqThreads * kSlot;   // 80 KB
+constexpr int kSmemBytes = kStages * kBStage + kRingBytes + 1024 /*barriers*/ + 1024 /*align*/;
 
 struct GemmArgs {
   PackedView v;
@@ -82,12 +86,13 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
   return d;
 }
 
-__device__ __forceinline__ void umma_f16(uint32_t dtmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
+// D (tensor memory) += A (tensor memory) . B (shared memory descriptor)
+__device__ __forceinline__ void umma_f16_ts(uint32_t dtmem, uint32_t atmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(dtmem),
+      "r"(atmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -114,6 +119,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// This thread's lane of the warp's TMEM quarter, 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
@@ -122,11 +138,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-__device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
 // ---- cp.async (per-thread asynchronous copies into shared memory) ----
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+template <int kBytes>
+__device__ __forceinline__ void cp_async(void* dst, const void* src) {
+  if constexpr (kBytes == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(smem_addr(dst)), "l"(src), "n"(kBytes)
+                 : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -152,34 +171,62 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// ---- exact dequantisation of 32 consecutive codes of one row (from shared memory) ----
+// ---- one row's 128-code group: copy its two 32-code pieces of half h ----
+// Piece j (stage 2g + j of the group) holds codes [64 j + 32 h, 64 j + 32 h + 32):
+// 4b bytes at byte 8 b j + 4 b h of the group (16 b bytes from the row start
+// times g); it lands at byte 32 j of the thread's ring slot.
+template <int B>
+__device__ __forceinline__ void copy_pieces(uint8_t* slot, const uint8_t* grp, int h) {
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const uint8_t* src = grp + 8 * B * j + 4 * B * h;
+    uint8_t* dst = slot + 32 * j;
+    if constexpr (B == 4) {
+      cp_async<16>(dst, src);
+    } else if constexpr (B == 8) {
+      cp_async<16>(dst, src);
+      cp_async<16>(dst + 16, src + 16);
+    } else if constexpr (B == 6) {
+#pragma unroll
+      for (int i = 0; i < 3; ++i) cp_async<8>(dst + 8 * i, src + 8 * i);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 3; ++i) cp_async<4>(dst + 4 * i, src + 4 * i);
+    }
+  }
+}
+
+__device__ __forceinline__ void copy_pieces_any(int b, uint8_t* slot, const uint8_t* grp, int h) {
+  switch (b) {
+    case 3: copy_pieces<3>(slot, grp, h); break;
+    case 4: copy_pieces<4>(slot, grp, h); break;
+    case 6: copy_pieces<6>(slot, grp, h); break;
+    default: copy_pieces<8>(slot, grp, h); break;
+  }
+}
+
+// ---- exact dequantisation of one 32-code piece (from the thread's ring slot) ----
 // q -> fp32 exactly through the bit pattern 2^23 + q (0x4B000000 | q) minus
 // 2^23; then t = q - z and p = s * t, each rounded to nearest in fp32 (the same
 // operations as dequant_exact, two lanes per instruction), then fp16.
 template <int B>
-__device__ __forceinline__ void dequant32(const uint8_t* row, int r, int o, float s, float z, uint32_t (&out)[16]) {
-  // row: this row's 128-byte slot line; o: byte offset of the 32 codes in the row
+__device__ __forceinline__ void dequant_piece(const uint8_t* piece, float s, float z, uint32_t (&out)[16]) {
   uint32_t w[B + 1];
-  const int sw = r & 7;
   if constexpr (B == 8 || B == 4) {
 #pragma unroll
     for (int i = 0; i < B / 4; ++i) {
-      const uint4 v = *reinterpret_cast<const uint4*>(row + ((((o >> 4) + i) ^ sw) << 4));
+      const uint4 v = *reinterpret_cast<const uint4*>(piece + 16 * i);
       w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
     }
   } else if constexpr (B == 6) {
 #pragma unroll
     for (int i = 0; i < 3; ++i) {
-      const int oo = o + 8 * i;
-      const uint2 v = *reinterpret_cast<const uint2*>(row + (((oo >> 4) ^ sw) << 4) + (oo & 15));
+      const uint2 v = *reinterpret_cast<const uint2*>(piece + 8 * i);
       w[2 * i] = v.x; w[2 * i + 1] = v.y;
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 3; ++i) {
-      const int oo = o + 4 * i;
-      w[i] = *reinterpret_cast<const uint32_t*>(row + (((oo >> 4) ^ sw) << 4) + (oo & 15));
-    }
+    for (int i = 0; i < 3; ++i) w[i] = *reinterpret_cast<const uint32_t*>(piece + 4 * i);
   }
   w[B] = 0;
   constexpr uint32_t kMask = (1u << B) - 1u;
@@ -207,13 +254,12 @@ __device__ __forceinline__ void dequant32(const uint8_t* row, int r, int o, floa
   }
 }
 
-__device__ __forceinline__ void dequant32_any(int b, const uint8_t* row, int r, int o, float s, float z,
-                                              uint32_t (&out)[16]) {
+__device__ __forceinline__ void dequant_piece_any(int b, const uint8_t* piece, float s, float z, uint32_t (&out)[16]) {
   switch (b) {
-    case 3: dequant32<3>(row, r, o, s, z, out); break;
-    case 4: dequant32<4>(row, r, o, s, z, out); break;
-    case 6: dequant32<6>(row, r, o, s, z, out); break;
-    default: dequant32<8>(row, r, o, s, z, out); break;
+    case 3: dequant_piece<3>(piece, s, z, out); break;
+    case 4: dequant_piece<4>(piece, s, z, out); break;
+    case 6: dequant_piece<6>(piece, s, z, out); break;
+    default: dequant_piece<8>(piece, s, z, out); break;
   }
 }
 
@@ -221,16 +267,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                                                               const __grid_constant__ GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint8_t* As = smem;
-  uint8_t* Bs = smem + kStages * kAStage;
-  uint8_t* Cs = Bs + kStages * kBStage;  // code ring
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Cs + kCodeRing * kCodeSlotBytes);
+  uint8_t* Bs = smem;
+  uint8_t* ring = Bs + kStages * kBStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kRingBytes);
   uint64_t* st_empty = bars;
   uint64_t* a_full = bars + kStages;
   uint64_t* b_full = bars + 2 * kStages;
   uint64_t* acc_full = bars + 3 * kStages;
-  uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles = a.m_tiles * a.n_tiles;
@@ -241,10 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       mbar_init(&a_full[s], kDeqWarps);
       mbar_init(&b_full[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
-    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -277,25 +320,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     if (lane == 0) {
       // kind::f16, fp32 accumulate, fp16 A and B, both K-major, M = 128, N = BN.
       const uint32_t idesc = (1u << 4) | ((uint32_t)(a.BN >> 3) << 17) | ((uint32_t)(kBMw >> 4) << 24);
+      const uint32_t dtmem = tmem_base + kAccCol;
       int g = 0, i = 0;
       for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
-        const int abuf = i & 1, ua = i >> 1;
-        if (ua > 0) wait_or_fail(&acc_empty[abuf], (ua - 1) & 1, 2u);
+        if (i > 0) wait_or_fail(acc_empty, (i - 1) & 1, 2u);
         tc_fence_after();
-        const uint32_t dtmem = tmem_base + (uint32_t)(abuf * kBNmax);
         for (int kb = 0; kb < a.KB; ++kb, ++g) {
           const int s = g % kStages, u = g / kStages;
           wait_or_fail(&a_full[s], u & 1, 4u);
           wait_or_fail(&b_full[s], u & 1, 8u);
           tc_fence_after();
-          const uint64_t ad = umma_desc_sw128(smem_addr(As + s * kAStage));
+          const uint32_t atmem = tmem_base + (uint32_t)(kACol + 32 * s);
           const uint64_t bd = umma_desc_sw128(smem_addr(Bs + s * kBStage));
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)  // 16 fp16 = 32 bytes = 2 descriptor units
-            umma_f16(dtmem, ad + 2u * k, bd + 2u * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < kBK / 16; ++k)  // 16 fp16 = 8 TMEM columns of A, 32 bytes = 2 descriptor units of B
+            umma_f16_ts(dtmem, atmem + 8u * k, bd + 2u * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
           umma_commit(&st_empty[s]);
         }
-        umma_commit(&acc_full[abuf]);
+        umma_commit(acc_full);
       }
     }
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
@@ -305,13 +347,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
       const int m0 = (t % a.m_tiles) * a.BN;
       const int n0 = (t / a.m_tiles) * kBMw;
-      const int abuf = i & 1, ua = i >> 1;
-      wait_or_fail(&acc_full[abuf], ua & 1, 16u);
+      wait_or_fail(acc_full, i & 1, 16u);
       tc_fence_after();
       const int n = n0 + 32 * q + lane;
       for (int c0 = 0; c0 < a.BN; c0 += 32) {
         uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(abuf * kBNmax + c0), r);
+        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCol + c0), r);
         if (n < a.v.N) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -322,53 +363,45 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[abuf]);
+      if (lane == 0) mbar_arrive(acc_empty);
     }
   } else if (warp >= kDeqWarp0) {
     // ---------------------------------------------------- dequantisation --
-    // Per 128-code group of the tile, all 256 threads copy the tile's codes
-    // (16-byte pieces, consecutive threads on consecutive pieces of a row) one
-    // group ahead into the code ring, then thread (r, h) dequantises row r,
-    // codes [32h, 32h + 32) of each of the group's two 64-code MMA stages.
-    const int dt = threadIdx.x - kDeqWarp0 * 32;  // 0..255
-    const int r = dt >> 1, h = dt & 1;
+    const int j = warp - kDeqWarp0;
+    const int q = j & 3, h = j >> 2;    // TMEM lane quarter (warp % 4) and half of each stage
+    const int r = 32 * q + lane;        // this thread's weight row in the tile
+    const int dt = threadIdx.x - kDeqWarp0 * 32;
     const int G = a.v.K / kGroup;
-    // copy cursor: tile ct, group cg
-    int ct = blockIdx.x, cg = 0;
-    const uint8_t* cbase[2] = {nullptr, nullptr};
-    int cb[2] = {4, 4}, cvalid = 0;
-    auto copy_tile = [&]() {
-      if (ct >= tiles) return;
-      const int n0 = (ct / a.m_tiles) * kBMw;
-      cvalid = min(kBMw, a.v.N - n0);
-      for (int hh = 0; hh < 2; ++hh)
-        if (64 * hh < cvalid) cbase[hh] = reinterpret_cast<const uint8_t*>(row_of(a.v, n0 + 64 * hh, cb[hh]));
+    const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kACol + 16 * h);
+    const int my_tiles = (tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int items = my_tiles * G;     // (tile, group) pairs of this CTA, in order
+    // copy cursor (item ci): the row pointer and width of this thread's row in tile ct
+    int ci = 0, ct = blockIdx.x, cg = 0, cb = 4;
+    const uint8_t* crow = nullptr;
+    auto set_copy_tile = [&]() {
+      const int n = (ct / a.m_tiles) * kBMw + r;
+      crow = nullptr;
+      if (ct < tiles && n < a.v.N) crow = reinterpret_cast<const uint8_t*>(row_of(a.v, n, cb));
     };
-    auto issue_group = [&](int slot) {
-      if (ct < tiles) {
-        uint8_t* dst = Cs + slot * kCodeSlotBytes;
-        const int P0 = 64 * cb[0], P = P0 + (cvalid > 64 ? 64 * cb[1] : 0);
-        for (int i = dt; i < P; i += kDeqThreads) {
-          const int hh = i >= P0 ? 1 : 0;
-          const int ii = i - hh * P0, bb = cb[hh];
-          const int rr = ii / bb, c = ii - rr * bb;
-          const int row = 64 * hh + rr;
-          if (row < cvalid) {
-            const uint8_t* src = cbase[hh] + (size_t)rr * (size_t)(a.v.K / 8 * bb) + (size_t)cg * 16 * bb + 16 * c;
-            cp_async16(dst + row * 128 + ((c ^ (row & 7)) << 4), src);
-          }
-        }
+    auto issue = [&]() {  // copies of item ci into ring slot ci % kRing, one commit group
+      if (ci < items && crow != nullptr)
+        copy_pieces_any(cb, ring + (size_t)(ci % kRing) * kDeqThreads * kSlot + dt * kSlot,
+                        crow + (size_t)cg * 16 * cb, h);
+      cp_async_commit();
+      if (ci < items) {
+        ++ci;
         if (++cg == G) {
           cg = 0;
           ct += gridDim.x;
-          copy_tile();
+          set_copy_tile();
         }
       }
-      cp_async_commit();
     };
-    copy_tile();
-    issue_group(0);
-    int q = 0, g = 0;
+    set_copy_tile();
+#pragma unroll 1
+    for (int k = 0; k < kRing - 1; ++k) issue();
+    int g = 0;  // pipeline stage counter (two stages per item)
+    int it = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int n = (t / a.m_tiles) * kBMw + r;
       const bool valid = n < a.v.N;
@@ -377,36 +410,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const __half* srow = a.scales + (size_t)n * G;
       const __half* zrow = a.zeros + (size_t)n * G;
       float sc = valid ? __half2float(srow[0]) : 0.f, zc = valid ? __half2float(zrow[0]) : 0.f;
-      for (int gi = 0; gi < G; ++gi, ++q) {
-        // next group's scale and zero (loaded now, used one group later)
-        float sn = 0.f, zn = 0.f;
+      for (int gi = 0; gi < G; ++gi, ++it) {
+        issue();                    // item it + kRing - 1
+        cp_async_wait<kRing - 1>();  // this thread's copies of item `it` have landed
+        float sn = 0.f, zn = 0.f;   // next group's scale and zero (used one group later)
         if (valid && gi + 1 < G) {
           sn = __half2float(srow[gi + 1]);
           zn = __half2float(zrow[gi + 1]);
         }
-        cp_async_wait<0>();            // this thread's copies of group q have landed
-        named_barrier(2, kDeqThreads);  // everyone's have; everyone is done with group q - 1
-        issue_group((q + 1) % kCodeRing);
-        const uint8_t* crow = Cs + (q % kCodeRing) * kCodeSlotBytes + r * 128;
+        const uint8_t* slot = ring + (size_t)(it % kRing) * kDeqThreads * kSlot + dt * kSlot;
 #pragma unroll 1
-        for (int j = 0; j < 2; ++j, ++g) {
+        for (int jj = 0; jj < 2; ++jj, ++g) {
           const int s = g % kStages, u = g / kStages;
           uint32_t out[16];
           if (valid) {
-            dequant32_any(b, crow, r, (8 * j + 4 * h) * b, sc, zc, out);
+            dequant_piece_any(b, slot + 32 * jj, sc, zc, out);
           } else {
 #pragma unroll
             for (int i2 = 0; i2 < 16; ++i2) out[i2] = 0u;
           }
           if (u > 0) wait_or_fail(&st_empty[s], (u - 1) & 1, 32u);
-          uint8_t* arow = As + s * kAStage + r * 128;
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            const int c = 4 * h + jj;
-            *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) =
-                make_uint4(out[4 * jj], out[4 * jj + 1], out[4 * jj + 2], out[4 * jj + 3]);
-          }
-          fence_async_shared();
+          tc_fence_after();
+          tmem_st16(tq + (uint32_t)(32 * s), out);
+          tmem_st_wait();
+          tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&a_full[s]);
         }
@@ -447,13 +474,9 @@ EncodeTiledFn encode_fn() {
 
 size_t gemm_workspace_bytes(int M, int K) { return ((size_t)M * K * 2 + 255) & ~(size_t)255; }
 
-qlin_status launch_gemm(const PackedView& v, const __half* scales, const __half* zeros,
-                        const uint32_t* sign_bits, const __half* x, __half* y, int M,
-                        void* workspace, cudaStream_t s) {
-  __half* xr = static_cast<__half*>(workspace);
-  qlin_status r = launch_rht(x, xr, sign_bits, M, v.K, s);
-  if (r != QLIN_OK) return r;
-
+// The GEMM proper, on activations already rotated into xr (M x K fp16).
+qlin_status launch_gemm_rotated(const PackedView& v, const __half* scales, const __half* zeros, const __half* xr,
+                                __half* y, int M, cudaStream_t s) {
   GemmArgs a;
   a.v = v;
   a.scales = scales;
@@ -472,7 +495,7 @@ qlin_status launch_gemm(const PackedView& v, const __half* scales, const __half*
   const cuuint64_t strides[1] = {(cuuint64_t)v.K * 2};
   const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)a.BN};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xr, dims, strides, box, estr,
+  CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(xr), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return record_cuda(cudaErrorInvalidValue);
@@ -490,6 +513,15 @@ qlin_status launch_gemm(const PackedView& v, const __half* scales, const __half*
   const int grid = std::min(tiles, 148);
   gemm_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(map, a);
   return record_cuda(cudaGetLastError());
+}
+
+qlin_status launch_gemm(const PackedView& v, const __half* scales, const __half* zeros,
+                        const uint32_t* sign_bits, const __half* x, __half* y, int M,
+                        void* workspace, cudaStream_t s) {
+  __half* xr = static_cast<__half*>(workspace);
+  qlin_status r = launch_rht(x, xr, sign_bits, M, v.K, s);
+  if (r != QLIN_OK) return r;
+  return launch_gemm_rotated(v, scales, zeros, xr, y, M, s);
 }
 
 unsigned take_gemm_error() {
@@ -588,30 +620,6 @@ extern "C" qlin_status qlin_gemm_noalloc(const qlin_desc* d, const void* packed,
   r = launch_rht(reinterpret_cast<const __half*>(x), xr, sign_bits, M, v.K, s);
   if (r != QLIN_OK) return r;
 
-  GemmArgs a;
-  a.v = v;
-  a.scales = reinterpret_cast<const __half*>(scales);
-  a.zeros = reinterpret_cast<const __half*>(zeros);
-  a.y = reinterpret_cast<__half*>(y);
-  a.M = M;
-  a.BN = std::min(kBNmax, (M + 15) / 16 * 16);
-  a.m_tiles = (M + a.BN - 1) / a.BN;
-  a.n_tiles = (v.N + kBMw - 1) / kBMw;
-  a.KB = v.K / kBK;
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return record_cuda(cudaErrorNotSupported);
-  CUtensorMap map;
-  const cuuint64_t dims[2] = {(cuuint64_t)v.K, (cuuint64_t)M};
-  const cuuint64_t strides[1] = {(cuuint64_t)v.K * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)a.BN};
-  const cuuint32_t estr[2] = {1, 1};
-  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
-      CUDA_SUCCESS)
-    return record_cuda(cudaErrorInvalidValue);
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) return record_cuda(e);
-  const int tiles = a.m_tiles * a.n_tiles;
-  gemm_tc_kernel<<<std::min(tiles, 148), kThreads, kSmemBytes, s>>>(map, a);
-  return record_cuda(cudaGetLastError());
+  return launch_gemm_rotated(v, reinterpret_cast<const __half*>(scales), reinterpret_cast<const __half*>(zeros),
+                             xr, reinterpret_cast<__half*>(y), M, s);
 }
