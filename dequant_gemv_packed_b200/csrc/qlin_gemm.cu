@@ -19,11 +19,12 @@
 // Warp roles: 0 TMA producer, 1 MMA issuer (one thread) and TMEM owner,
 // 4..7 epilogue (TMEM lane quarters 0..3), 8..15 dequantisation.
 // Dequantisation warp 8 + j owns TMEM lane quarter q = j % 4 (weight rows
-// 32q .. 32q+31 of the tile, one per thread) and half h = j / 4 of every
-// 64-code stage.  Each thread copies its own row's two 32-code pieces of every
-// 128-code group kRing groups ahead (cp.async into a private ring slot), so the
-// dequantisation warps never wait for one another; results go to tensor memory,
-// which the MMA reads without a proxy fence.
+// 32q .. 32q+31 of the tile, one per thread) and the stages of parity h = j / 4
+// (codes [64h, 64h + 64) of every 128-code group).  Each thread copies its own
+// row's 64-code piece and the group's scale and zero kRing groups ahead
+// (16-byte cp.async into a private ring slot), so the dequantisation warps
+// never wait for one another; results go to tensor memory, which the MMA reads
+// without a proxy fence.
 // The weight tile is the MMA's M side because dequantisation costs ALU work
 // per weight element per activation tile: with 256 activation rows per tile
 // each weight element is dequantised once per 256 rows of X.
@@ -54,7 +55,7 @@ constexpr int kTmemCols = 512;
 constexpr int kAccCol = 0;     // accumulator: columns [0, BN)
 constexpr int kACol = 256;     // A of stage s: columns [kACol + 32 s, kACol + 32 s + 32)
 constexpr int kRing = 4;       // 128-code groups in flight per dequantisation thread
-constexpr int kSlot = 80;      // bytes per thread per group: pieces at 0 and 32 (16-byte stride 5: no bank conflicts)
+constexpr int kSlot = 80;      // bytes per thread per group: piece at 0, scale/zero pairs at 64/68 (stride 5 x 16 B: no bank conflicts)
 constexpr int kRingBytes = kRing * kDeqThreads * kSlot;   // 80 KB
 constexpr int kSmemBytes = kStages * kBStage + kRingBytes + 1024 /*barriers*/ + 1024 /*align*/;
 
@@ -119,13 +120,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// This thread's lane of the warp's TMEM quarter, 16 consecutive 32-bit columns.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+// This thread's lane of the warp's TMEM quarter, 32 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -171,54 +175,40 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// ---- one row's 128-code group: copy its two 32-code pieces of half h ----
-// Piece j (stage 2g + j of the group) holds codes [64 j + 32 h, 64 j + 32 h + 32):
-// 4b bytes at byte 8 b j + 4 b h of the group (16 b bytes from the row start
-// times g); it lands at byte 32 j of the thread's ring slot.
+// ---- one row's 128-code group: copy its 64-code piece of parity h ----
+// The piece holds codes [64 h, 64 h + 64): 8b bytes at byte 8 b h of the group
+// (16 b bytes per group from the row start); it lands at byte 0 of the
+// thread's ring slot.  The 4-byte words holding the group's scale and zero
+// (fp16 pairs, aligned) land at bytes 64 and 68.
 template <int B>
-__device__ __forceinline__ void copy_pieces(uint8_t* slot, const uint8_t* grp, int h) {
+__device__ __forceinline__ void copy_piece(uint8_t* slot, const uint8_t* grp, int h) {
+  const uint8_t* src = grp + 8 * B * h;
+  if constexpr (B == 3) {
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const uint8_t* src = grp + 8 * B * j + 4 * B * h;
-    uint8_t* dst = slot + 32 * j;
-    if constexpr (B == 4) {
-      cp_async<16>(dst, src);
-    } else if constexpr (B == 8) {
-      cp_async<16>(dst, src);
-      cp_async<16>(dst + 16, src + 16);
-    } else if constexpr (B == 6) {
+    for (int i = 0; i < 3; ++i) cp_async<8>(slot + 8 * i, src + 8 * i);
+  } else {
 #pragma unroll
-      for (int i = 0; i < 3; ++i) cp_async<8>(dst + 8 * i, src + 8 * i);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 3; ++i) cp_async<4>(dst + 4 * i, src + 4 * i);
-    }
+    for (int i = 0; i < B / 2; ++i) cp_async<16>(slot + 16 * i, src + 16 * i);
   }
 }
 
-__device__ __forceinline__ void copy_pieces_any(int b, uint8_t* slot, const uint8_t* grp, int h) {
+__device__ __forceinline__ void copy_piece_any(int b, uint8_t* slot, const uint8_t* grp, int h) {
   switch (b) {
-    case 3: copy_pieces<3>(slot, grp, h); break;
-    case 4: copy_pieces<4>(slot, grp, h); break;
-    case 6: copy_pieces<6>(slot, grp, h); break;
-    default: copy_pieces<8>(slot, grp, h); break;
+    case 3: copy_piece<3>(slot, grp, h); break;
+    case 4: copy_piece<4>(slot, grp, h); break;
+    case 6: copy_piece<6>(slot, grp, h); break;
+    default: copy_piece<8>(slot, grp, h); break;
   }
 }
 
-// ---- exact dequantisation of one 32-code piece (from the thread's ring slot) ----
+// ---- exact dequantisation of one 64-code piece (from the thread's ring slot) ----
 // q -> fp32 exactly through the bit pattern 2^23 + q (0x4B000000 | q) minus
 // 2^23; then t = q - z and p = s * t, each rounded to nearest in fp32 (the same
 // operations as dequant_exact, two lanes per instruction), then fp16.
 template <int B>
-__device__ __forceinline__ void dequant_piece(const uint8_t* piece, float s, float z, uint32_t (&out)[16]) {
-  uint32_t w[B + 1];
-  if constexpr (B == 8 || B == 4) {
-#pragma unroll
-    for (int i = 0; i < B / 4; ++i) {
-      const uint4 v = *reinterpret_cast<const uint4*>(piece + 16 * i);
-      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-    }
-  } else if constexpr (B == 6) {
+__device__ __forceinline__ void dequant_piece(const uint8_t* piece, float s, float z, uint32_t (&out)[32]) {
+  uint32_t w[2 * B + 1];
+  if constexpr (B == 3) {
 #pragma unroll
     for (int i = 0; i < 3; ++i) {
       const uint2 v = *reinterpret_cast<const uint2*>(piece + 8 * i);
@@ -226,13 +216,16 @@ __device__ __forceinline__ void dequant_piece(const uint8_t* piece, float s, flo
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 3; ++i) w[i] = *reinterpret_cast<const uint32_t*>(piece + 4 * i);
+    for (int i = 0; i < B / 2; ++i) {
+      const uint4 v = *reinterpret_cast<const uint4*>(piece + 16 * i);
+      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+    }
   }
-  w[B] = 0;
+  w[2 * B] = 0;
   constexpr uint32_t kMask = (1u << B) - 1u;
   const uint64_t c23 = pk2(8388608.0f, 8388608.0f), zz = pk2(z, z), ss = pk2(s, s);
 #pragma unroll
-  for (int i = 0; i < 32; i += 2) {
+  for (int i = 0; i < 64; i += 2) {
     uint32_t m[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -254,13 +247,19 @@ __device__ __forceinline__ void dequant_piece(const uint8_t* piece, float s, flo
   }
 }
 
-__device__ __forceinline__ void dequant_piece_any(int b, const uint8_t* piece, float s, float z, uint32_t (&out)[16]) {
+__device__ __forceinline__ void dequant_piece_any(int b, const uint8_t* piece, float s, float z, uint32_t (&out)[32]) {
   switch (b) {
     case 3: dequant_piece<3>(piece, s, z, out); break;
     case 4: dequant_piece<4>(piece, s, z, out); break;
     case 6: dequant_piece<6>(piece, s, z, out); break;
     default: dequant_piece<8>(piece, s, z, out); break;
   }
+}
+
+// fp16 element `idx` of an array, from the aligned 4-byte word holding it.
+__device__ __forceinline__ float half_of_pair(uint32_t word, int idx) {
+  const uint16_t bits = (idx & 1) ? (uint16_t)(word >> 16) : (uint16_t)(word & 0xFFFFu);
+  return __half2float(__ushort_as_half(bits));
 }
 
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap,
@@ -283,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&st_empty[s], 1);
-      mbar_init(&a_full[s], kDeqWarps);
+      mbar_init(&a_full[s], kDeqWarps / 2);  // one warp per lane quarter writes each stage
       mbar_init(&b_full[s], 1);
     }
     mbar_init(acc_full, 1);
@@ -368,25 +367,33 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   } else if (warp >= kDeqWarp0) {
     // ---------------------------------------------------- dequantisation --
     const int j = warp - kDeqWarp0;
-    const int q = j & 3, h = j >> 2;    // TMEM lane quarter (warp % 4) and half of each stage
+    const int q = j & 3, h = j >> 2;    // TMEM lane quarter (warp % 4) and stage parity
     const int r = 32 * q + lane;        // this thread's weight row in the tile
     const int dt = threadIdx.x - kDeqWarp0 * 32;
     const int G = a.v.K / kGroup;
-    const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kACol + 16 * h);
+    const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)kACol;
     const int my_tiles = (tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     const int items = my_tiles * G;     // (tile, group) pairs of this CTA, in order
-    // copy cursor (item ci): the row pointer and width of this thread's row in tile ct
+    // copy cursor (item ci): this thread's row in tile ct, its width and scale/zero row
     int ci = 0, ct = blockIdx.x, cg = 0, cb = 4;
     const uint8_t* crow = nullptr;
+    size_t csz = 0;
     auto set_copy_tile = [&]() {
       const int n = (ct / a.m_tiles) * kBMw + r;
       crow = nullptr;
-      if (ct < tiles && n < a.v.N) crow = reinterpret_cast<const uint8_t*>(row_of(a.v, n, cb));
+      if (ct < tiles && n < a.v.N) {
+        crow = reinterpret_cast<const uint8_t*>(row_of(a.v, n, cb));
+        csz = (size_t)n * G;
+      }
     };
     auto issue = [&]() {  // copies of item ci into ring slot ci % kRing, one commit group
-      if (ci < items && crow != nullptr)
-        copy_pieces_any(cb, ring + (size_t)(ci % kRing) * kDeqThreads * kSlot + dt * kSlot,
-                        crow + (size_t)cg * 16 * cb, h);
+      if (ci < items && crow != nullptr) {
+        uint8_t* slot = ring + (size_t)(ci % kRing) * kDeqThreads * kSlot + dt * kSlot;
+        copy_piece_any(cb, slot, crow + (size_t)cg * 16 * cb, h);
+        const size_t e = (csz + cg) & ~(size_t)1;
+        cp_async<4>(slot + 64, a.scales + e);
+        cp_async<4>(slot + 68, a.zeros + e);
+      }
       cp_async_commit();
       if (ci < items) {
         ++ci;
@@ -400,45 +407,35 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     set_copy_tile();
 #pragma unroll 1
     for (int k = 0; k < kRing - 1; ++k) issue();
-    int g = 0;  // pipeline stage counter (two stages per item)
     int it = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int n = (t / a.m_tiles) * kBMw + r;
       const bool valid = n < a.v.N;
       int b = 4;
       if (valid) (void)row_of(a.v, n, b);
-      const __half* srow = a.scales + (size_t)n * G;
-      const __half* zrow = a.zeros + (size_t)n * G;
-      float sc = valid ? __half2float(srow[0]) : 0.f, zc = valid ? __half2float(zrow[0]) : 0.f;
       for (int gi = 0; gi < G; ++gi, ++it) {
-        issue();                    // item it + kRing - 1
+        issue();                     // item it + kRing - 1
         cp_async_wait<kRing - 1>();  // this thread's copies of item `it` have landed
-        float sn = 0.f, zn = 0.f;   // next group's scale and zero (used one group later)
-        if (valid && gi + 1 < G) {
-          sn = __half2float(srow[gi + 1]);
-          zn = __half2float(zrow[gi + 1]);
-        }
         const uint8_t* slot = ring + (size_t)(it % kRing) * kDeqThreads * kSlot + dt * kSlot;
-#pragma unroll 1
-        for (int jj = 0; jj < 2; ++jj, ++g) {
-          const int s = g % kStages, u = g / kStages;
-          uint32_t out[16];
-          if (valid) {
-            dequant_piece_any(b, slot + 32 * jj, sc, zc, out);
-          } else {
+        const int g = 2 * it + h;    // pipeline stage of this piece
+        const int s = g % kStages, u = g / kStages;
+        uint32_t out[32];
+        if (valid) {
+          const int e = (int)(((size_t)n * G + gi) & 1);
+          const float sc = half_of_pair(*reinterpret_cast<const uint32_t*>(slot + 64), e);
+          const float zc = half_of_pair(*reinterpret_cast<const uint32_t*>(slot + 68), e);
+          dequant_piece_any(b, slot, sc, zc, out);
+        } else {
 #pragma unroll
-            for (int i2 = 0; i2 < 16; ++i2) out[i2] = 0u;
-          }
-          if (u > 0) wait_or_fail(&st_empty[s], (u - 1) & 1, 32u);
-          tc_fence_after();
-          tmem_st16(tq + (uint32_t)(32 * s), out);
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&a_full[s]);
+          for (int i2 = 0; i2 < 32; ++i2) out[i2] = 0u;
         }
-        sc = sn;
-        zc = zn;
+        if (u > 0) wait_or_fail(&st_empty[s], (u - 1) & 1, 32u);
+        tc_fence_after();
+        tmem_st32(tq + (uint32_t)(32 * s), out);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[s]);
       }
     }
     cp_async_wait<0>();
