@@ -55,6 +55,7 @@ constexpr int kTmemCols = 512;
 constexpr int kAccCol = 0;     // accumulator: columns [0, BN)
 constexpr int kACol = 256;     // A of stage s: columns [kACol + 32 s, kACol + 32 s + 32)
 constexpr int kRing = 4;       // 128-code groups in flight per dequantisation thread
+constexpr int kSms = 148;
 constexpr int kSlot = 80;      // bytes per thread per group: piece at 0, scale/zero pairs at 64/68 (stride 5 x 16 B: no bank conflicts)
 constexpr int kRingBytes = kRing * kDeqThreads * kSlot;   // 80 KB
 constexpr int kSmemBytes = kStages * kBStage + kRingBytes + 1024 /*barriers*/ + 1024 /*align*/;
@@ -65,7 +66,51 @@ struct GemmArgs {
   const __half* zeros;
   __half* y;
   int M, BN, m_tiles, n_tiles, KB;
+  // Stream-K schedule (stream_k != 0): CTA c takes the 128-code groups
+  // [c T / P, (c+1) T / P) of the T = tiles * G (tile, group) pairs in tile
+  // order, P = gridDim.x.  A tile split between CTAs is finished by the CTA
+  // holding its first groups, which adds the other CTAs' fp32 partial sums
+  // (partials[c]: [BN][128], flag[c] = 1 when written) in CTA order.
+  int stream_k;
+  uint32_t* flags;   // [P], zero on entry (cleared by the rotation kernel), zero on exit
+  float* partials;   // [P][part_cols][128]
+  int part_cols;     // BN rounded up to the 32 columns one TMEM load covers
 };
+
+// The (tile, group range) segments one CTA works through, in order.
+struct Segments {
+  int G, tiles, stream_k;
+  long long it, end;  // stream-K: group cursor and end
+  int t;              // data-parallel: tile cursor
+  __device__ void init(const GemmArgs& a) {
+    G = a.v.K / kGroup;
+    tiles = a.m_tiles * a.n_tiles;
+    stream_k = a.stream_k;
+    const long long T = (long long)tiles * G, P = gridDim.x;
+    it = T * blockIdx.x / P;
+    end = T * (blockIdx.x + 1) / P;
+    t = blockIdx.x;
+  }
+  // Next segment: tile t, groups [g0, g1); false when done.
+  __device__ bool next(int& tile, int& g0, int& g1) {
+    if (!stream_k) {
+      if (t >= tiles) return false;
+      tile = t;
+      g0 = 0;
+      g1 = G;
+      t += gridDim.x;
+      return true;
+    }
+    if (it >= end) return false;
+    tile = (int)(it / G);
+    g0 = (int)(it % G);
+    g1 = (int)min((long long)G, g0 + (end - it));
+    it += g1 - g0;
+    return true;
+  }
+};
+
+__device__ __forceinline__ long long sk_start(long long T, int P, int c) { return T * c / P; }
 
 __device__ __forceinline__ void gemm_fail(unsigned code) { atomicOr(&g_gemm_error, code); }
 
@@ -303,10 +348,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
-      int g = 0;
-      for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+      int g = 0, t, g0, g1;
+      Segments sg;
+      sg.init(a);
+      while (sg.next(t, g0, g1)) {
         const int m0 = (t % a.m_tiles) * a.BN;
-        for (int kb = 0; kb < a.KB; ++kb, ++g) {
+        for (int kb = 2 * g0; kb < 2 * g1; ++kb, ++g) {
           const int s = g % kStages, u = g / kStages;
           if (u > 0) wait_or_fail(&st_empty[s], (u - 1) & 1, 1u);
           mbar_arrive_expect_tx(&b_full[s], (uint32_t)a.BN * kBK * 2);
@@ -320,11 +367,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       // kind::f16, fp32 accumulate, fp16 A and B, both K-major, M = 128, N = BN.
       const uint32_t idesc = (1u << 4) | ((uint32_t)(a.BN >> 3) << 17) | ((uint32_t)(kBMw >> 4) << 24);
       const uint32_t dtmem = tmem_base + kAccCol;
-      int g = 0, i = 0;
-      for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      int g = 0, i = 0, t, g0, g1;
+      Segments sg;
+      sg.init(a);
+      for (; sg.next(t, g0, g1); ++i) {
         if (i > 0) wait_or_fail(acc_empty, (i - 1) & 1, 2u);
         tc_fence_after();
-        for (int kb = 0; kb < a.KB; ++kb, ++g) {
+        for (int kb = 2 * g0; kb < 2 * g1; ++kb, ++g) {
           const int s = g % kStages, u = g / kStages;
           wait_or_fail(&a_full[s], u & 1, 4u);
           wait_or_fail(&b_full[s], u & 1, 8u);
@@ -333,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           const uint64_t bd = umma_desc_sw128(smem_addr(Bs + s * kBStage));
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)  // 16 fp16 = 8 TMEM columns of A, 32 bytes = 2 descriptor units of B
-            umma_f16_ts(dtmem, atmem + 8u * k, bd + 2u * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            umma_f16_ts(dtmem, atmem + 8u * k, bd + 2u * k, idesc, (kb > 2 * g0 || k > 0) ? 1u : 0u);
           umma_commit(&st_empty[s]);
         }
         umma_commit(acc_full);
@@ -342,22 +391,77 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
     // --------------------------------------------------------- epilogue --
     const int q = warp & 3;  // TMEM lanes 32q..32q+31 = weight rows of the tile
-    int i = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+    const int row = 32 * q + lane;
+    const long long T = (long long)tiles * (a.v.K / kGroup);
+    const int G = a.v.K / kGroup, P = gridDim.x, c = blockIdx.x;
+    int i = 0, t, g0, g1;
+    Segments sg;
+    sg.init(a);
+    for (; sg.next(t, g0, g1); ++i) {
       const int m0 = (t % a.m_tiles) * a.BN;
       const int n0 = (t / a.m_tiles) * kBMw;
+      const int n = n0 + row;
       wait_or_fail(acc_full, i & 1, 16u);
       tc_fence_after();
-      const int n = n0 + 32 * q + lane;
-      for (int c0 = 0; c0 < a.BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCol + c0), r);
-        if (n < a.v.N) {
+      if (g0 > 0) {
+        // a later part of a split tile: hand the fp32 partial to the tile's owner
+        float* dst = a.partials + (size_t)c * a.part_cols * kBMw + row;
+        for (int c0 = 0; c0 < a.BN; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCol + c0), r);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int m = m0 + c0 + j;
-            if (m < a.M) a.y[(size_t)m * a.v.N + n] = __float2half_rn(__uint_as_float(r[j]));
+          for (int j = 0; j < 32; ++j) dst[(size_t)(c0 + j) * kBMw] = __uint_as_float(r[j]);
+        }
+        __threadfence();
+        named_barrier(3, 128);
+        if (q == 0 && lane == 0)
+          asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a.flags + c), "r"(1u) : "memory");
+      } else {
+        // the tile's contributors after this CTA (stream-K split): CTAs whose
+        // groups overlap [g1, G) of this tile
+        int c_last = c;
+        if (g1 < G)
+          while (c_last + 1 < P && sk_start(T, P, c_last + 1) < (long long)(t + 1) * G) ++c_last;
+        for (int cc = c + 1; cc <= c_last; ++cc) {
+          if (lane == 0) {
+            uint32_t f = 0;
+            const uint64_t t0 = globaltimer_ns();
+            while (true) {
+              asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(f) : "l"(a.flags + cc) : "memory");
+              if (f || g_gemm_error) break;
+              if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                gemm_fail(64u);
+                break;
+              }
+            }
           }
+          __syncwarp();
+          // acquire in every lane before its loads of the partial
+          asm volatile("{\n\t.reg .b32 f;\n\tld.acquire.gpu.global.u32 f, [%0];\n\t}" ::"l"(a.flags + cc) : "memory");
+        }
+        for (int c0 = 0; c0 < a.BN; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCol + c0), r);
+          float acc[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(r[j]);
+          for (int cc = c + 1; cc <= c_last; ++cc) {
+            const float* src = a.partials + (size_t)cc * a.part_cols * kBMw + (size_t)c0 * kBMw + row;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[j] += __ldcg(src + (size_t)j * kBMw);
+          }
+          if (n < a.v.N) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int m = m0 + c0 + j;
+              if (m < a.M) a.y[(size_t)m * a.v.N + n] = __float2half_rn(acc[j]);
+            }
+          }
+        }
+        if (c_last > c) {
+          named_barrier(3, 128);  // every epilogue warp has read the partials
+          if (q == 0 && lane == 0)
+            for (int cc = c + 1; cc <= c_last; ++cc) a.flags[cc] = 0u;
         }
       }
       tc_fence_before();
@@ -372,22 +476,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int dt = threadIdx.x - kDeqWarp0 * 32;
     const int G = a.v.K / kGroup;
     const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)kACol;
-    const int my_tiles = (tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-    const int items = my_tiles * G;     // (tile, group) pairs of this CTA, in order
-    // copy cursor (item ci): this thread's row in tile ct, its width and scale/zero row
-    int ci = 0, ct = blockIdx.x, cg = 0, cb = 4;
+    // copy cursor: the (tile, group) items of this CTA's segments, in order;
+    // this thread's row in tile ct, its width and its scale/zero row
+    Segments cs;
+    cs.init(a);
+    int ct = 0, cg = 0, cg1 = 0, cb = 4;
+    bool cmore = cs.next(ct, cg, cg1);
     const uint8_t* crow = nullptr;
     size_t csz = 0;
+    int ci = 0;
     auto set_copy_tile = [&]() {
       const int n = (ct / a.m_tiles) * kBMw + r;
       crow = nullptr;
-      if (ct < tiles && n < a.v.N) {
+      if (cmore && n < a.v.N) {
         crow = reinterpret_cast<const uint8_t*>(row_of(a.v, n, cb));
         csz = (size_t)n * G;
       }
     };
     auto issue = [&]() {  // copies of item ci into ring slot ci % kRing, one commit group
-      if (ci < items && crow != nullptr) {
+      if (cmore && crow != nullptr) {
         uint8_t* slot = ring + (size_t)(ci % kRing) * kDeqThreads * kSlot + dt * kSlot;
         copy_piece_any(cb, slot, crow + (size_t)cg * 16 * cb, h);
         const size_t e = (csz + cg) & ~(size_t)1;
@@ -395,11 +502,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         cp_async<4>(slot + 68, a.zeros + e);
       }
       cp_async_commit();
-      if (ci < items) {
+      if (cmore) {
         ++ci;
-        if (++cg == G) {
-          cg = 0;
-          ct += gridDim.x;
+        if (++cg == cg1) {
+          cmore = cs.next(ct, cg, cg1);
           set_copy_tile();
         }
       }
@@ -407,13 +513,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     set_copy_tile();
 #pragma unroll 1
     for (int k = 0; k < kRing - 1; ++k) issue();
-    int it = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+    int it = 0, t, g0, g1;
+    Segments sg;
+    sg.init(a);
+    while (sg.next(t, g0, g1)) {
       const int n = (t / a.m_tiles) * kBMw + r;
       const bool valid = n < a.v.N;
       int b = 4;
       if (valid) (void)row_of(a.v, n, b);
-      for (int gi = 0; gi < G; ++gi, ++it) {
+      for (int gi = g0; gi < g1; ++gi, ++it) {
         issue();                     // item it + kRing - 1
         cp_async_wait<kRing - 1>();  // this thread's copies of item `it` have landed
         const uint8_t* slot = ring + (size_t)(it % kRing) * kDeqThreads * kSlot + dt * kSlot;
@@ -469,11 +577,25 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-size_t gemm_workspace_bytes(int M, int K) { return ((size_t)M * K * 2 + 255) & ~(size_t)255; }
+// Workspace of qlin_gemm: the rotated activations, then the stream-K
+// completion flags and partial sums.
+struct GemmWorkspace {
+  size_t xr_bytes, flags_off, part_off, total;
+  GemmWorkspace(int M, int K) {
+    const int BN = std::min(kBNmax, (M + 15) / 16 * 16);
+    xr_bytes = ((size_t)M * K * 2 + 255) & ~(size_t)255;
+    flags_off = xr_bytes;
+    part_off = flags_off + 1024;
+    total = part_off + (size_t)kSms * ((BN + 31) & ~31) * kBMw * 4;
+  }
+};
+
+size_t gemm_workspace_bytes(int M, int K) { return GemmWorkspace(M, K).total; }
 
 // The GEMM proper, on activations already rotated into xr (M x K fp16).
+// flags/partials: the stream-K scratch (both null: one CTA per tile instead).
 qlin_status launch_gemm_rotated(const PackedView& v, const __half* scales, const __half* zeros, const __half* xr,
-                                __half* y, int M, cudaStream_t s) {
+                                __half* y, int M, cudaStream_t s, uint32_t* flags, float* partials) {
   GemmArgs a;
   a.v = v;
   a.scales = scales;
@@ -484,6 +606,10 @@ qlin_status launch_gemm_rotated(const PackedView& v, const __half* scales, const
   a.m_tiles = (M + a.BN - 1) / a.BN;
   a.n_tiles = (v.N + kBMw - 1) / kBMw;
   a.KB = v.K / kBK;
+  a.stream_k = flags != nullptr ? 1 : 0;
+  a.part_cols = (a.BN + 31) & ~31;
+  a.flags = flags;
+  a.partials = partials;
 
   EncodeTiledFn enc = encode_fn();
   if (!enc) return record_cuda(cudaErrorNotSupported);
@@ -506,8 +632,9 @@ qlin_status launch_gemm_rotated(const PackedView& v, const __half* scales, const
     if (e != cudaSuccess) return record_cuda(e);
     if (dev < 64) configured |= 1ull << dev;
   }
-  const int tiles = a.m_tiles * a.n_tiles;
-  const int grid = std::min(tiles, 148);
+  const long long tiles = (long long)a.m_tiles * a.n_tiles;
+  const long long work = a.stream_k ? tiles * (v.K / kGroup) : tiles;
+  const int grid = (int)std::min<long long>(work, kSms);
   gemm_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(map, a);
   return record_cuda(cudaGetLastError());
 }
@@ -515,10 +642,14 @@ qlin_status launch_gemm_rotated(const PackedView& v, const __half* scales, const
 qlin_status launch_gemm(const PackedView& v, const __half* scales, const __half* zeros,
                         const uint32_t* sign_bits, const __half* x, __half* y, int M,
                         void* workspace, cudaStream_t s) {
-  __half* xr = static_cast<__half*>(workspace);
-  qlin_status r = launch_rht(x, xr, sign_bits, M, v.K, s);
+  const GemmWorkspace ws(M, v.K);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  __half* xr = reinterpret_cast<__half*>(base);
+  uint32_t* flags = reinterpret_cast<uint32_t*>(base + ws.flags_off);
+  float* partials = reinterpret_cast<float*>(base + ws.part_off);
+  qlin_status r = launch_rht(x, xr, sign_bits, M, v.K, s, flags, kSms);
   if (r != QLIN_OK) return r;
-  return launch_gemm_rotated(v, scales, zeros, xr, y, M, s);
+  return launch_gemm_rotated(v, scales, zeros, xr, y, M, s, flags, partials);
 }
 
 unsigned take_gemm_error() {
@@ -618,5 +749,5 @@ extern "C" qlin_status qlin_gemm_noalloc(const qlin_desc* d, const void* packed,
   if (r != QLIN_OK) return r;
 
   return launch_gemm_rotated(v, reinterpret_cast<const __half*>(scales), reinterpret_cast<const __half*>(zeros),
-                             xr, reinterpret_cast<__half*>(y), M, s);
+                             xr, reinterpret_cast<__half*>(y), M, s, nullptr, nullptr);
 }

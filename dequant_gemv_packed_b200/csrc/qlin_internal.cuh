@@ -42,8 +42,10 @@ qlin_status launch_pack(const PackedView& v, const uint8_t* codes, uint8_t* pack
 qlin_status launch_unpack(const PackedView& v, uint8_t* codes, cudaStream_t s);
 qlin_status launch_dequant(const PackedView& v, const __half* scales, const __half* zeros,
                            __half* w, cudaStream_t s);
+// Rotation of M rows of x into xr; also zeroes clear[0, nclear) (completion
+// flags of the kernel that follows on the stream).
 qlin_status launch_rht(const __half* x, __half* xr, const uint32_t* sign_bits, int M, int K,
-                       cudaStream_t s);
+                       cudaStream_t s, uint32_t* clear = nullptr, int nclear = 0);
 size_t gemv_workspace_bytes(int bits, int N, int K, int M);
 unsigned take_gemv_error();
 unsigned take_gemm_error();

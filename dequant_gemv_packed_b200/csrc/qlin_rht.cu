@@ -11,8 +11,11 @@
 namespace qlin {
 
 __global__ void rht_kernel(const __half* __restrict__ x, __half* __restrict__ xr,
-                           const uint32_t* __restrict__ sign_bits, int M, int K) {
+                           const uint32_t* __restrict__ sign_bits, int M, int K, uint32_t* clear, int nclear) {
   const int lane = threadIdx.x & 31;
+  // Words the kernel that follows expects to find zero (its completion flags).
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nclear; i += blockDim.x) clear[i] = 0u;
   const int blocks_per_row = K / kHadamard;
   const long long total = (long long)M * blocks_per_row;
   const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -40,12 +43,12 @@ __global__ void rht_kernel(const __half* __restrict__ x, __half* __restrict__ xr
 }
 
 qlin_status launch_rht(const __half* x, __half* xr, const uint32_t* sign_bits, int M, int K,
-                       cudaStream_t s) {
+                       cudaStream_t s, uint32_t* clear, int nclear) {
   const long long warps = (long long)M * (K / kHadamard);
   const int threads = 256;
   long long blocks = (warps * 32 + threads - 1) / threads;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  rht_kernel<<<(int)blocks, threads, 0, s>>>(x, xr, sign_bits, M, K);
+  rht_kernel<<<(int)blocks, threads, 0, s>>>(x, xr, sign_bits, M, K, clear, nclear);
   return record_cuda(cudaGetLastError());
 }
 

@@ -259,6 +259,23 @@ def test_gemm_ragged(bits, N, K, M):
     assert Q.qlin_device_error() == 0
 
 
+@pytest.mark.parametrize("N,K,M", [(9728, 2560, 256), (77, 384, 1), (1000, 1280, 600)])
+def test_gemm_deterministic_split_tiles(N, K, M):
+    """Tiles split between CTAs are summed in a fixed order: repeated calls are
+    bit-identical (and match the oracle)."""
+    w = _rand_weight(N, K, 6, seed=N + 7)
+    a = W.draw_activation(M, K, seed=3).to(DEV)
+    d, packed = packed_on_device(w)
+    y1 = Q.qlin_gemm(d, packed, w.scales, w.zeros, a.sign_bits, a.x)
+    y2 = Q.qlin_gemm(d, packed, w.scales, w.zeros, a.sign_bits, a.x)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    rows = sample_rows(N, 64, seed=1) if N > 2000 else None
+    got = y1 if rows is None else y1[:, torch.as_tensor(rows, device=y1.device)]
+    assert_close(got, oracle_rows(w, a, rows), f"gemm split N{N} K{K} M{M}")
+    assert Q.qlin_device_error() == 0
+
+
 def test_gemm_matches_gemv_at_m16():
     w, a = W.down(M=16, device=DEV)
     d, packed = packed_on_device(w)
