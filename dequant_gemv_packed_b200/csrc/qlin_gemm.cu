@@ -54,11 +54,12 @@ constexpr int kEpiWarp0 = 4;
 constexpr int kTmemCols = 512;
 constexpr int kAccCol = 0;     // accumulator: columns [0, BN)
 constexpr int kACol = 256;     // A of stage s: columns [kACol + 32 s, kACol + 32 s + 32)
-constexpr int kRing = 4;       // 128-code groups in flight per dequantisation thread
+constexpr int kRing = 3;       // 128-code groups in flight per dequantisation thread
 constexpr int kSms = 148;
 constexpr int kSlot = 80;      // bytes per thread per group: piece at 0, scale/zero pairs at 64/68 (stride 5 x 16 B: no bank conflicts)
 constexpr int kRingBytes = kRing * kDeqThreads * kSlot;   // 80 KB
-constexpr int kSmemBytes = kStages * kBStage + kRingBytes + 1024 /*barriers*/ + 1024 /*align*/;
+constexpr int kStageOut = 128 * kBMw * 2;                // Y staging: up to 128 activation rows x 128 weight rows, fp16
+constexpr int kSmemBytes = kStages * kBStage + kRingBytes + kStageOut + 1024 /*barriers*/ + 1024 /*align*/;
 
 struct GemmArgs {
   PackedView v;
@@ -75,6 +76,8 @@ struct GemmArgs {
   uint32_t* flags;   // [P], zero on entry (cleared by the rotation kernel), zero on exit
   float* partials;   // [P][part_cols][128]
   int part_cols;     // BN rounded up to the 32 columns one TMEM load covers
+  int tma_store;     // Y written by TMA tensor stores through shared memory (N % 8 == 0)
+  int box_m;         // activation rows per store box: min(BN, 128)
 };
 
 // The (tile, group range) segments one CTA works through, in order.
@@ -186,6 +189,19 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
       : "memory");
 }
+
+// Tensor store of a shared-memory box to global memory (out-of-range parts are
+// not written), and the waits on such stores.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_addr(src)), "r"(x), "r"(y)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ---- cp.async (per-thread asynchronous copies into shared memory) ----
 template <int kBytes>
@@ -308,12 +324,14 @@ __device__ __forceinline__ float half_of_pair(uint32_t word, int idx) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                              const __grid_constant__ CUtensorMap ymap,
                                                               const __grid_constant__ GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* Bs = smem;
   uint8_t* ring = Bs + kStages * kBStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kRingBytes);
+  __half* ystage = reinterpret_cast<__half*>(ring + kRingBytes);  // [box_m][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kRingBytes + kStageOut);
   uint64_t* st_empty = bars;
   uint64_t* a_full = bars + kStages;
   uint64_t* b_full = bars + 2 * kStages;
@@ -417,6 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         if (q == 0 && lane == 0)
           asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a.flags + c), "r"(1u) : "memory");
       } else {
+        if (a.tma_store) {  // the staging buffer may still be read by the previous tile's store
+          if (q == 0 && lane == 0) tma_store_wait_read();
+          named_barrier(3, 128);
+        }
         // the tile's contributors after this CTA (stream-K split): CTAs whose
         // groups overlap [g1, G) of this tile
         int c_last = c;
@@ -450,7 +472,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 #pragma unroll
             for (int j = 0; j < 32; ++j) acc[j] += __ldcg(src + (size_t)j * kBMw);
           }
-          if (n < a.v.N) {
+          if (a.tma_store) {
+            // a box of box_m activation rows: stage it (fp16, [m][n]), then one thread stores it
+            const int cb = c0 % a.box_m;
+            if (cb == 0 && c0 > 0) {  // the previous box of this tile is in flight: wait for its reads
+              if (q == 0 && lane == 0) tma_store_wait_read();
+              named_barrier(3, 128);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (cb + j < a.box_m) ystage[(cb + j) * kBMw + row] = __float2half_rn(acc[j]);
+            if (cb + 32 >= a.box_m || c0 + 32 >= a.BN) {
+              fence_async_shared();
+              named_barrier(3, 128);
+              if (q == 0 && lane == 0) tma_store_2d(&ymap, ystage, n0, m0 + c0 - cb);
+            }
+          } else if (n < a.v.N) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int m = m0 + c0 + j;
@@ -468,6 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
     }
+    if (a.tma_store && q == 0 && lane == 0) tma_store_wait_all();
   } else if (warp >= kDeqWarp0) {
     // ---------------------------------------------------- dequantisation --
     const int j = warp - kDeqWarp0;
@@ -622,6 +660,20 @@ qlin_status launch_gemm_rotated(const PackedView& v, const __half* scales, const
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return record_cuda(cudaErrorInvalidValue);
+  // Y [M][N] fp16: tensor stores need rows of a multiple of 16 bytes
+  CUtensorMap ymap;
+  a.box_m = std::min(a.BN, 128);
+  a.tma_store = (v.N % 8 == 0) ? 1 : 0;
+  if (a.tma_store) {
+    const cuuint64_t ydims[2] = {(cuuint64_t)v.N, (cuuint64_t)M};
+    const cuuint64_t ystrides[1] = {(cuuint64_t)v.N * 2};
+    const cuuint32_t ybox[2] = {(cuuint32_t)kBMw, (cuuint32_t)a.box_m};
+    cr = enc(&ymap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, y, ydims, ystrides, ybox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return record_cuda(cudaErrorInvalidValue);
+  } else {
+    ymap = map;  // unused
+  }
 
   static unsigned long long configured = 0;
   int dev = 0;
@@ -635,7 +687,7 @@ qlin_status launch_gemm_rotated(const PackedView& v, const __half* scales, const
   const long long tiles = (long long)a.m_tiles * a.n_tiles;
   const long long work = a.stream_k ? tiles * (v.K / kGroup) : tiles;
   const int grid = (int)std::min<long long>(work, kSms);
-  gemm_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(map, a);
+  gemm_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(map, ymap, a);
   return record_cuda(cudaGetLastError());
 }
 
