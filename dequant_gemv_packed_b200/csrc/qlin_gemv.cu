@@ -41,8 +41,7 @@
 //     weight before waiting on the previous kernel, and waits only before it
 //     reads x; two CTAs fit on an SM, so the next call's weight stream runs
 //     under this call's arithmetic.
-// Other cases (M > 1, mixed widths): the activation rotation runs as its own
-// kernel into the workspace, then gemv_simple_kernel.
+// Other cases (M > 1, mixed widths, very long K): gemv_mma_kernel below.
 #include <algorithm>
 
 #include "qlin_internal.cuh"
@@ -818,40 +817,210 @@ qlin_status launch_gemv1(const Args& a, cudaStream_t s) {
   }
 }
 
-// ----------------------------------------------------- general fallback --
+// ------------------------------------------- M up to 16: tensor cores ----
+//
+// gemv_mma_kernel: rotation of x by the stand-alone kernel into the workspace
+// (with each 128-value group's sum), then one warp per share of the (16-row
+// tile, 128-code group) items.  Per item the codes become the A operand of
+// m16n8k16 products (q exact in fp16: the code in the mantissa of 1024.0, minus
+// 1024), the rotated x the B operand (n8 = 8 rows of x per product), fp32
+// accumulation; the group's scale and zero then apply to the accumulator,
+// y += s (sum q x - z sum x).  Thread (g, t) = (lane / 4, lane % 4) takes codes
+// [32t, 32t + 32) of the group for weight rows g and g + 8 (k-step j: codes
+// 32t + 4j .. 32t + 4j + 3 in k slots 2t, 2t+1, 2t+8, 2t+9), and the same
+// codes' x for x row g: both operands use one permutation of k, so the sum is
+// unchanged.  Partial sums of a row tile split between warps go to the
+// workspace; the last warp to finish the tile adds them in warp order
+// (deterministic) and writes y.
 
-// One warp per weight row; the rotated activations come from the workspace.
-__global__ void gemv_simple_kernel(PackedView v, const __half* __restrict__ scales,
-                                   const __half* __restrict__ zeros,
-                                   const __half* __restrict__ xr, __half* __restrict__ y, int M) {
-  const int lane = threadIdx.x & 31;
-  const int warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int nwarps = (gridDim.x * blockDim.x) >> 5;
-  const int G = v.K / kGroup;
-  for (int n = warp0; n < v.N; n += nwarps) {
-    int b;
-    const uint32_t* row = row_of(v, n, b);
-    float acc[16];
+struct MmaArgs {
+  PackedView v;
+  const __half* scales;
+  const __half* zeros;
+  const __half* xr;     // [M][K] rotated x
+  const float* xsum;    // [M][G] group sums of xr
+  __half* y;            // [M][N]
+  float* part;          // [W * max_seg][16][16]
+  uint32_t* counters;   // [tiles], zero on entry, zero on exit
+  int M, G, tiles, max_seg;
+  long long T;          // tiles * G items
+};
+
+// Code i (0..31) of a 32-code run held in words w (b bits each, little-endian).
+template <int B>
+__device__ __forceinline__ uint32_t run_code(const uint32_t (&w)[B], int i) {
+  const int bit = B * i;
+  const int wi = bit >> 5, sh = bit & 31;
+  uint32_t v = w[wi] >> sh;
+  if (sh + B > 32) v |= w[wi + 1 < B ? wi + 1 : wi] << (32 - sh);
+  return v & ((1u << B) - 1u);
+}
+
+// (q_i, q_{i+1}) as two exact fp16 values.
+template <int B>
+__device__ __forceinline__ uint32_t code_pair(const uint32_t (&w)[B], int i) {
+  const uint32_t h = (run_code<B>(w, i) | (run_code<B>(w, i + 1) << 16)) | kMagic;
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&h), __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// The 32-code run [32t, 32t + 32) of group g of a row: 4b bytes.
+template <int B>
+__device__ __forceinline__ void load_run(const uint32_t* row, int g, int t, uint32_t (&w)[B]) {
+  const uint32_t* p = row + (size_t)g * 4 * B + t * B;  // 16b bytes per group, 4b per run
+  if constexpr (B == 4) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (B == 8) {
+    const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(p)), v1 = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w; w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+  } else if constexpr (B == 6) {
 #pragma unroll
-    for (int m = 0; m < 16; ++m) acc[m] = 0.f;
-    for (int k = lane; k < v.K; k += 32) {
-      const int g = k / kGroup;
-      const float s = __half2float(scales[(size_t)n * G + g]);
-      const float z = __half2float(zeros[(size_t)n * G + g]);
-      const float w = __half2float(dequant_exact(code_at(row, b, k), s, z));
-#pragma unroll
-      for (int m = 0; m < 16; ++m)
-        if (m < M) acc[m] = fmaf(w, __half2float(xr[(size_t)m * v.K + k]), acc[m]);
+    for (int i = 0; i < 3; ++i) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p) + i);
+      w[2 * i] = v.x; w[2 * i + 1] = v.y;
     }
+  } else {
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      if (m >= M) break;
-      float a = acc[m];
+    for (int i = 0; i < B; ++i) w[i] = __ldg(p + i);
+  }
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+               "{%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// sum_k q x over one group for rows ra, rb of width B and x rows 8 nt + g:
+// d[nt][0..3] = (ra, 2t), (ra, 2t+1), (rb, 2t), (rb, 2t+1) of column tile nt.
+template <int B, int NT>
+__device__ __forceinline__ void group_products(const uint32_t* row_a, const uint32_t* row_b, int grp, int t,
+                                               const uint2* const (&xp)[NT], float (&d)[NT][4]) {
+  uint32_t wa[B], wb[B];
+  load_run<B>(row_a, grp, t, wa);
+  load_run<B>(row_b, grp, t, wb);
 #pragma unroll
-      for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      if (lane == 0) y[(size_t)m * v.N + n] = __float2half_rn(a);
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[nt][i] = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t a0 = code_pair<B>(wa, 4 * j), a2 = code_pair<B>(wa, 4 * j + 2);
+    const uint32_t a1 = code_pair<B>(wb, 4 * j), a3 = code_pair<B>(wb, 4 * j + 2);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint2 xv = __ldg(xp[nt] + j);  // x of codes 32t + 4j .. 32t + 4j + 3
+      mma16816(d[nt], a0, a1, a2, a3, xv.x, xv.y);
     }
   }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(256) gemv_mma_kernel(const __grid_constant__ MmaArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int gq = lane >> 2, t = lane & 3;
+  const long long W = (long long)gridDim.x * (blockDim.x >> 5);
+  const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const long long i0 = a.T * w / W, i1 = a.T * (w + 1) / W;
+  if (i0 >= i1) return;
+  const int N = a.v.N, K = a.v.K, G = a.G, M = a.M;
+  const int rt_first = (int)(i0 / G);
+  // x rows of this lane's B fragments (zero beyond M)
+  const int xm[2] = {gq, 8 + gq};
+  float acc[NT][4];
+  int cur = -1;
+  auto flush = [&](int rt) {
+    // this warp's partial of row tile rt: rows 16 rt + {gq, gq + 8}, x rows 8 nt + {2t, 2t + 1}
+    const int seg = rt - rt_first;
+    float* slot = a.part + ((size_t)w * a.max_seg + seg) * 256;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      slot[gq * 16 + 8 * nt + 2 * t] = acc[nt][0];
+      slot[gq * 16 + 8 * nt + 2 * t + 1] = acc[nt][1];
+      slot[(gq + 8) * 16 + 8 * nt + 2 * t] = acc[nt][2];
+      slot[(gq + 8) * 16 + 8 * nt + 2 * t + 1] = acc[nt][3];
+    }
+    __threadfence();
+    __syncwarp();
+    // warps covering tile rt: the ones holding its first and last items
+    const long long f = (long long)rt * G, l = f + G - 1;
+    // warp of item i: the largest w' with T w' / W <= i
+    auto warp_of = [&](long long i) {
+      long long lo = 0, hi = W - 1;
+      while (lo < hi) {
+        const long long mid = (lo + hi + 1) >> 1;
+        if (a.T * mid / W <= i) lo = mid; else hi = mid - 1;
+      }
+      return lo;
+    };
+    const long long w_first = warp_of(f), w_last = warp_of(l);
+    unsigned prev = 0;
+    if (lane == 0) prev = atomicAdd(a.counters + rt, 1u);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (prev != (unsigned)(w_last - w_first)) return;  // not the last contributor
+    __threadfence();
+    // sum the contributors' partials in warp order and write y
+    float sum[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sum[e] = 0.f;
+    for (long long ww = w_first; ww <= w_last; ++ww) {
+      const int sg = rt - (int)(a.T * ww / W / G);
+      const float* sl = a.part + ((size_t)ww * a.max_seg + sg) * 256;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sum[e] += __ldcg(sl + lane * 8 + e);
+    }
+    // element lane * 8 + e of the 16 x 16 tile: weight row r = (lane*8+e) / 16, x row m = (lane*8+e) % 16
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int idx = lane * 8 + e, r = 16 * rt + idx / 16, m = idx % 16;
+      if (r < N && m < M) a.y[(size_t)m * N + r] = __float2half_rn(sum[e]);
+    }
+    if (lane == 0) a.counters[rt] = 0u;  // ready for the next call
+  };
+  for (long long i = i0; i < i1; ++i) {
+    const int rt = (int)(i / G), grp = (int)(i % G);
+    if (rt != cur) {
+      if (cur >= 0) flush(cur);
+      cur = rt;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+    }
+    const int ra = min(16 * rt + gq, N - 1), rb = min(16 * rt + gq + 8, N - 1);
+    int b = 4, bb = 4;
+    const uint32_t* row_a = row_of(a.v, ra, b);
+    const uint32_t* row_b = row_of(a.v, rb, bb);  // same 64-row block as row a: same width
+    const uint2* xp[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int m = min(xm[nt], M - 1);
+      xp[nt] = reinterpret_cast<const uint2*>(a.xr + (size_t)m * K + (size_t)grp * kGroup + 32 * t);
+    }
+    float d[NT][4];
+    switch (b) {
+      case 3: group_products<3, NT>(row_a, row_b, grp, t, xp, d); break;
+      case 4: group_products<4, NT>(row_a, row_b, grp, t, xp, d); break;
+      case 6: group_products<6, NT>(row_a, row_b, grp, t, xp, d); break;
+      default: group_products<8, NT>(row_a, row_b, grp, t, xp, d); break;
+    }
+    const float sa = __half2float(a.scales[(size_t)ra * G + grp]), za = __half2float(a.zeros[(size_t)ra * G + grp]);
+    const float sb = __half2float(a.scales[(size_t)rb * G + grp]), zb = __half2float(a.zeros[(size_t)rb * G + grp]);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int m0 = 8 * nt + 2 * t;
+      const float x0 = m0 < M ? a.xsum[(size_t)m0 * G + grp] : 0.f;
+      const float x1 = m0 + 1 < M ? a.xsum[(size_t)(m0 + 1) * G + grp] : 0.f;
+      acc[nt][0] += sa * fmaf(-za, x0, d[nt][0]);
+      acc[nt][1] += sa * fmaf(-za, x1, d[nt][1]);
+      acc[nt][2] += sb * fmaf(-zb, x0, d[nt][2]);
+      acc[nt][3] += sb * fmaf(-zb, x1, d[nt][3]);
+    }
+  }
+  flush(cur);
 }
 
 }  // namespace
@@ -861,11 +1030,33 @@ static bool gemv_fused_path(int bits, int N, int K, int M) {
   return M == 1 && bits != 0 && make_plan(bits, N, K, p);
 }
 
+// Workspace of the tensor-core path: rotated x, its group sums, the row-tile
+// counters and the warps' partial sums.
+struct MmaWorkspace {
+  size_t xsum_off, cnt_off, part_off, total;
+  int tiles, warps, max_seg, grid, warps_per_block;
+  MmaWorkspace(int N, int K, int M) {
+    const int G = K / kGroup;
+    tiles = (N + 15) / 16;
+    const long long T = (long long)tiles * G;
+    // no more warps than items: every warp then owns at least one item (and
+    // reports to each row tile it touches)
+    warps_per_block = (int)std::min<long long>(8, T);
+    grid = (int)std::max<long long>(1, std::min<long long>(kSms, T / warps_per_block));
+    warps = grid * warps_per_block;
+    const long long per = (T + warps - 1) / warps;
+    max_seg = (int)((per + G - 1) / G) + 1;
+    xsum_off = ((size_t)M * K * 2 + 255) & ~(size_t)255;
+    cnt_off = xsum_off + (((size_t)M * G * 4 + 255) & ~(size_t)255);
+    part_off = cnt_off + (((size_t)tiles * 4 + 255) & ~(size_t)255);
+    total = part_off + (size_t)warps * max_seg * 256 * 4;
+  }
+};
+
 size_t gemv_workspace_bytes(int bits, int N, int K, int M) {
-  // The fused M = 1 kernel rotates x in its prologue and needs no workspace;
-  // the other cases rotate x into the workspace first.
+  // The fused M = 1 kernel rotates x in its prologue and needs no workspace.
   if (gemv_fused_path(bits, N, K, M)) return 0;
-  return ((size_t)M * K * 2 + 255) & ~(size_t)255;
+  return MmaWorkspace(N, K, M).total;
 }
 
 qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half* zeros,
@@ -891,13 +1082,29 @@ qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half*
       }
     }
   }
-  __half* xr = static_cast<__half*>(workspace);
-  qlin_status r = launch_rht(x, xr, sign_bits, M, v.K, s);
+  const MmaWorkspace ws(v.N, v.K, M);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  MmaArgs a;
+  a.v = v;
+  a.scales = scales;
+  a.zeros = zeros;
+  a.xr = reinterpret_cast<const __half*>(base);
+  a.xsum = reinterpret_cast<const float*>(base + ws.xsum_off);
+  a.y = y;
+  a.counters = reinterpret_cast<uint32_t*>(base + ws.cnt_off);
+  a.part = reinterpret_cast<float*>(base + ws.part_off);
+  a.M = M;
+  a.G = v.K / kGroup;
+  a.tiles = ws.tiles;
+  a.max_seg = ws.max_seg;
+  a.T = (long long)ws.tiles * a.G;
+  qlin_status r = launch_rht(x, reinterpret_cast<__half*>(base), sign_bits, M, v.K, s, a.counters, ws.tiles,
+                             reinterpret_cast<float*>(base + ws.xsum_off));
   if (r != QLIN_OK) return r;
-  const int threads = 256;
-  int blocks = (v.N * 32 + threads - 1) / threads;
-  if (blocks > 148 * 8) blocks = 148 * 8;
-  gemv_simple_kernel<<<blocks, threads, 0, s>>>(v, scales, zeros, xr, y, M);
+  if (M <= 8)
+    gemv_mma_kernel<1><<<ws.grid, 32 * ws.warps_per_block, 0, s>>>(a);
+  else
+    gemv_mma_kernel<2><<<ws.grid, 32 * ws.warps_per_block, 0, s>>>(a);
   return record_cuda(cudaGetLastError());
 }
 

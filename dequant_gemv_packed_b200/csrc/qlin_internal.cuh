@@ -43,9 +43,10 @@ qlin_status launch_unpack(const PackedView& v, uint8_t* codes, cudaStream_t s);
 qlin_status launch_dequant(const PackedView& v, const __half* scales, const __half* zeros,
                            __half* w, cudaStream_t s);
 // Rotation of M rows of x into xr; also zeroes clear[0, nclear) (completion
-// flags of the kernel that follows on the stream).
+// flags of the kernel that follows on the stream) and, if xsum is given,
+// writes the sum of each row's 128-value blocks of xr: xsum[m * K/128 + block].
 qlin_status launch_rht(const __half* x, __half* xr, const uint32_t* sign_bits, int M, int K,
-                       cudaStream_t s, uint32_t* clear = nullptr, int nclear = 0);
+                       cudaStream_t s, uint32_t* clear = nullptr, int nclear = 0, float* xsum = nullptr);
 size_t gemv_workspace_bytes(int bits, int N, int K, int M);
 unsigned take_gemv_error();
 unsigned take_gemm_error();

@@ -11,7 +11,8 @@
 namespace qlin {
 
 __global__ void rht_kernel(const __half* __restrict__ x, __half* __restrict__ xr,
-                           const uint32_t* __restrict__ sign_bits, int M, int K, uint32_t* clear, int nclear) {
+                           const uint32_t* __restrict__ sign_bits, int M, int K, uint32_t* clear, int nclear,
+                           float* xsum) {
   const int lane = threadIdx.x & 31;
   // Words the kernel that follows expects to find zero (its completion flags).
   if (blockIdx.x == 0)
@@ -39,16 +40,22 @@ __global__ void rht_kernel(const __half* __restrict__ x, __half* __restrict__ xr
     out.x = *reinterpret_cast<uint32_t*>(&h01);
     out.y = *reinterpret_cast<uint32_t*>(&h23);
     *reinterpret_cast<uint2*>(xr + base) = out;
+    if (xsum) {  // sum of the block's rounded values (one group of 128 along K)
+      float sum = (__low2float(h01) + __high2float(h01)) + (__low2float(h23) + __high2float(h23));
+#pragma unroll
+      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if (lane == 0) xsum[t] = sum;
+    }
   }
 }
 
 qlin_status launch_rht(const __half* x, __half* xr, const uint32_t* sign_bits, int M, int K,
-                       cudaStream_t s, uint32_t* clear, int nclear) {
+                       cudaStream_t s, uint32_t* clear, int nclear, float* xsum) {
   const long long warps = (long long)M * (K / kHadamard);
   const int threads = 256;
   long long blocks = (warps * 32 + threads - 1) / threads;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  rht_kernel<<<(int)blocks, threads, 0, s>>>(x, xr, sign_bits, M, K, clear, nclear);
+  rht_kernel<<<(int)blocks, threads, 0, s>>>(x, xr, sign_bits, M, K, clear, nclear, xsum);
   return record_cuda(cudaGetLastError());
 }
 
