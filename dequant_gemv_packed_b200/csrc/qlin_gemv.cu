@@ -897,11 +897,8 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // sum_k q x over one group for rows ra, rb of width B and x rows 8 nt + g:
 // d[nt][0..3] = (ra, 2t), (ra, 2t+1), (rb, 2t), (rb, 2t+1) of column tile nt.
 template <int B, int NT>
-__device__ __forceinline__ void group_products(const uint32_t* row_a, const uint32_t* row_b, int grp, int t,
+__device__ __forceinline__ void group_products(const uint32_t (&wa)[B], const uint32_t (&wb)[B],
                                                const uint2* const (&xp)[NT], float (&d)[NT][4]) {
-  uint32_t wa[B], wb[B];
-  load_run<B>(row_a, grp, t, wa);
-  load_run<B>(row_b, grp, t, wb);
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -918,7 +915,7 @@ __device__ __forceinline__ void group_products(const uint32_t* row_a, const uint
   }
 }
 
-template <int NT>
+template <int B, int NT>
 __global__ void __launch_bounds__(256) gemv_mma_kernel(const __grid_constant__ MmaArgs a) {
   const int lane = threadIdx.x & 31;
   const int gq = lane >> 2, t = lane & 3;
@@ -947,15 +944,8 @@ __global__ void __launch_bounds__(256) gemv_mma_kernel(const __grid_constant__ M
     __syncwarp();
     // warps covering tile rt: the ones holding its first and last items
     const long long f = (long long)rt * G, l = f + G - 1;
-    // warp of item i: the largest w' with T w' / W <= i
-    auto warp_of = [&](long long i) {
-      long long lo = 0, hi = W - 1;
-      while (lo < hi) {
-        const long long mid = (lo + hi + 1) >> 1;
-        if (a.T * mid / W <= i) lo = mid; else hi = mid - 1;
-      }
-      return lo;
-    };
+    // warp of item i: the largest w' with floor(T w' / W) <= i, i.e. T w' < (i + 1) W
+    auto warp_of = [&](long long i) { return ((i + 1) * W - 1) / a.T; };
     const long long w_first = warp_of(f), w_last = warp_of(l);
     unsigned prev = 0;
     if (lane == 0) prev = atomicAdd(a.counters + rt, 1u);
@@ -980,8 +970,48 @@ __global__ void __launch_bounds__(256) gemv_mma_kernel(const __grid_constant__ M
     }
     if (lane == 0) a.counters[rt] = 0u;  // ready for the next call
   };
-  for (long long i = i0; i < i1; ++i) {
+  // The next item's code runs, scales and zeros are loaded while the current
+  // item is multiplied (one item of prefetch).
+  constexpr int kW = B ? B : 8;  // words of a 32-code run (mixed widths: up to 8)
+  uint32_t nwa[kW], nwb[kW];
+  int nb = B;
+  float nsa = 0.f, nza = 0.f, nsb = 0.f, nzb = 0.f;
+  auto fetch = [&](long long i) {
     const int rt = (int)(i / G), grp = (int)(i % G);
+    const int ra = min(16 * rt + gq, N - 1), rb = min(16 * rt + gq + 8, N - 1);
+    const uint32_t* row_a = row_of(a.v, ra, nb);
+    const uint32_t* row_b = row_of(a.v, rb, nb);  // same 64-row block: same width
+    if constexpr (B != 0) {
+      load_run<B>(row_a, grp, t, nwa);
+      load_run<B>(row_b, grp, t, nwb);
+    } else {
+      switch (nb) {
+        case 3:
+          load_run<3>(row_a, grp, t, reinterpret_cast<uint32_t(&)[3]>(nwa));
+          load_run<3>(row_b, grp, t, reinterpret_cast<uint32_t(&)[3]>(nwb));
+          break;
+        case 4:
+          load_run<4>(row_a, grp, t, reinterpret_cast<uint32_t(&)[4]>(nwa));
+          load_run<4>(row_b, grp, t, reinterpret_cast<uint32_t(&)[4]>(nwb));
+          break;
+        case 6:
+          load_run<6>(row_a, grp, t, reinterpret_cast<uint32_t(&)[6]>(nwa));
+          load_run<6>(row_b, grp, t, reinterpret_cast<uint32_t(&)[6]>(nwb));
+          break;
+        default:
+          load_run<8>(row_a, grp, t, nwa);
+          load_run<8>(row_b, grp, t, nwb);
+          break;
+      }
+    }
+    nsa = __half2float(a.scales[(size_t)ra * G + grp]);
+    nza = __half2float(a.zeros[(size_t)ra * G + grp]);
+    nsb = __half2float(a.scales[(size_t)rb * G + grp]);
+    nzb = __half2float(a.zeros[(size_t)rb * G + grp]);
+  };
+  fetch(i0);
+  int rt = (int)(i0 / G), grp = (int)(i0 % G);  // item i = rt * G + grp, advanced incrementally
+  for (long long i = i0; i < i1; ++i) {
     if (rt != cur) {
       if (cur >= 0) flush(cur);
       cur = rt;
@@ -990,10 +1020,15 @@ __global__ void __launch_bounds__(256) gemv_mma_kernel(const __grid_constant__ M
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
     }
-    const int ra = min(16 * rt + gq, N - 1), rb = min(16 * rt + gq + 8, N - 1);
-    int b = 4, bb = 4;
-    const uint32_t* row_a = row_of(a.v, ra, b);
-    const uint32_t* row_b = row_of(a.v, rb, bb);  // same 64-row block as row a: same width
+    uint32_t wa[kW], wb[kW];
+#pragma unroll
+    for (int e = 0; e < kW; ++e) {
+      wa[e] = nwa[e];
+      wb[e] = nwb[e];
+    }
+    const int bw = nb;
+    const float sa = nsa, za = nza, sb = nsb, zb = nzb;
+    if (i + 1 < i1) fetch(i + 1);
     const uint2* xp[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -1001,14 +1036,24 @@ __global__ void __launch_bounds__(256) gemv_mma_kernel(const __grid_constant__ M
       xp[nt] = reinterpret_cast<const uint2*>(a.xr + (size_t)m * K + (size_t)grp * kGroup + 32 * t);
     }
     float d[NT][4];
-    switch (b) {
-      case 3: group_products<3, NT>(row_a, row_b, grp, t, xp, d); break;
-      case 4: group_products<4, NT>(row_a, row_b, grp, t, xp, d); break;
-      case 6: group_products<6, NT>(row_a, row_b, grp, t, xp, d); break;
-      default: group_products<8, NT>(row_a, row_b, grp, t, xp, d); break;
+    if constexpr (B != 0) {
+      group_products<B, NT>(wa, wb, xp, d);
+    } else {
+      switch (bw) {
+        case 3:
+          group_products<3, NT>(reinterpret_cast<uint32_t(&)[3]>(wa), reinterpret_cast<uint32_t(&)[3]>(wb), xp, d);
+          break;
+        case 4:
+          group_products<4, NT>(reinterpret_cast<uint32_t(&)[4]>(wa), reinterpret_cast<uint32_t(&)[4]>(wb), xp, d);
+          break;
+        case 6:
+          group_products<6, NT>(reinterpret_cast<uint32_t(&)[6]>(wa), reinterpret_cast<uint32_t(&)[6]>(wb), xp, d);
+          break;
+        default:
+          group_products<8, NT>(wa, wb, xp, d);
+          break;
+      }
     }
-    const float sa = __half2float(a.scales[(size_t)ra * G + grp]), za = __half2float(a.zeros[(size_t)ra * G + grp]);
-    const float sb = __half2float(a.scales[(size_t)rb * G + grp]), zb = __half2float(a.zeros[(size_t)rb * G + grp]);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int m0 = 8 * nt + 2 * t;
@@ -1019,8 +1064,24 @@ __global__ void __launch_bounds__(256) gemv_mma_kernel(const __grid_constant__ M
       acc[nt][2] += sb * fmaf(-zb, x0, d[nt][2]);
       acc[nt][3] += sb * fmaf(-zb, x1, d[nt][3]);
     }
+    if (++grp == G) {
+      grp = 0;
+      ++rt;
+    }
   }
   flush(cur);
+}
+
+template <int B>
+void launch_mma(const MmaArgs& a, int grid, int threads, int M, cudaStream_t s) {
+  if (M <= 8)
+    gemv_mma_kernel<B, 1><<<grid, threads, 0, s>>>(a);
+  else
+    gemv_mma_kernel<B, 2><<<grid, threads, 0, s>>>(a);
+}
+
+void gemv_mma_mixed(const MmaArgs& a, int grid, int threads, int M, cudaStream_t s) {
+  launch_mma<0>(a, grid, threads, M, s);
 }
 
 }  // namespace
@@ -1101,10 +1162,16 @@ qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half*
   qlin_status r = launch_rht(x, reinterpret_cast<__half*>(base), sign_bits, M, v.K, s, a.counters, ws.tiles,
                              reinterpret_cast<float*>(base + ws.xsum_off));
   if (r != QLIN_OK) return r;
-  if (M <= 8)
-    gemv_mma_kernel<1><<<ws.grid, 32 * ws.warps_per_block, 0, s>>>(a);
-  else
-    gemv_mma_kernel<2><<<ws.grid, 32 * ws.warps_per_block, 0, s>>>(a);
+  if (v.bits == 0) {
+    gemv_mma_mixed(a, ws.grid, 32 * ws.warps_per_block, M, s);
+  } else {
+    switch (v.bits) {
+      case 3: launch_mma<3>(a, ws.grid, 32 * ws.warps_per_block, M, s); break;
+      case 4: launch_mma<4>(a, ws.grid, 32 * ws.warps_per_block, M, s); break;
+      case 6: launch_mma<6>(a, ws.grid, 32 * ws.warps_per_block, M, s); break;
+      default: launch_mma<8>(a, ws.grid, 32 * ws.warps_per_block, M, s); break;
+    }
+  }
   return record_cuda(cudaGetLastError());
 }
 
