@@ -899,6 +899,13 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 template <int B, int NT>
 __device__ __forceinline__ void group_products(const uint32_t (&wa)[B], const uint32_t (&wb)[B],
                                                const uint2* const (&xp)[NT], float (&d)[NT][4]) {
+  // all of the group's x fragments first (x of codes 32t + 4j .. 32t + 4j + 3), so
+  // that their loads overlap one another and the decoding
+  uint2 xv[NT][8];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) xv[nt][j] = __ldg(xp[nt] + j);
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -908,10 +915,7 @@ __device__ __forceinline__ void group_products(const uint32_t (&wa)[B], const ui
     const uint32_t a0 = code_pair<B>(wa, 4 * j), a2 = code_pair<B>(wa, 4 * j + 2);
     const uint32_t a1 = code_pair<B>(wb, 4 * j), a3 = code_pair<B>(wb, 4 * j + 2);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const uint2 xv = __ldg(xp[nt] + j);  // x of codes 32t + 4j .. 32t + 4j + 3
-      mma16816(d[nt], a0, a1, a2, a3, xv.x, xv.y);
-    }
+    for (int nt = 0; nt < NT; ++nt) mma16816(d[nt], a0, a1, a2, a3, xv[nt][j].x, xv[nt][j].y);
   }
 }
 
