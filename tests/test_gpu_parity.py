@@ -173,6 +173,16 @@ def test_gemv_m1_shapes(bits, N, K):
     _gemv_case(w, a, what=f"b{bits} N{N} K{K} M1")
 
 
+@pytest.mark.parametrize("bits", [3, 4, 6, 8])
+@pytest.mark.parametrize("N,K", [(4737, 1280), (5000, 1024), (6000, 1536), (4800, 4096), (5000, 128), (9728, 384)])
+def test_gemv_m1_tall_shapes(bits, N, K):
+    """M = 1 with 32 or more rows a CTA: several consumer iterations a chunk,
+    ragged last chunks, 1 to 10 consumer warps."""
+    w = _rand_weight(N, K, bits, seed=5 * N + bits)
+    a = W.draw_activation(1, K, seed=N + 2).to(DEV)
+    _gemv_case(w, a, what=f"b{bits} N{N} K{K} M1")
+
+
 def test_gemv_mixed():
     bb = [6, 8, 4, 3, 8]
     w = _rand_weight(64 * len(bb), 1280, 0, seed=5, block_bits=bb)
