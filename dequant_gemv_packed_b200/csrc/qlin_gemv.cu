@@ -67,7 +67,7 @@ constexpr int kPartialBudget = 24 * 1024;
 constexpr int kMaxStages = 16;
 constexpr int kSms = 148;
 
-template <int N> struct int_ {};
+template <int N> struct int_ { static constexpr int value = N; };
 
 // A unit is the run of codes one lane multiplies with its x registers.
 template <int B> struct UnitT;
@@ -627,26 +627,42 @@ __global__ void __launch_bounds__(kMaxThreads, 2) gemv1_kernel(const __grid_cons
     const __half* sp = s_ring + (size_t)s * p.sz_halves + aoff + g;
     const __half* zp = z_ring + (size_t)s * p.sz_halves + aoff + g;
     float* pchunk = part + (size_t)(wt * Rc) * NW + warp;
-    // R rows per iteration (independent accumulator chains).  Every lane runs
-    // every iteration (the row sums are warp shuffles); lanes whose row is at
-    // or past `cr` read the chunk's last row instead and store nothing.
-    for (int rb = 0; rb < cr; rb += R * RS) {
+    // One pass: RR rows a lane (independent accumulator chains), RR * RS rows
+    // a warp.  Every lane runs every pass (the row sums are warp shuffles);
+    // lanes whose row is at or past `cr` read the chunk's last row instead and
+    // store nothing.
+    const auto pass = [&](int rb, auto rows_tag) {
+      constexpr int RR = decltype(rows_tag)::value;
       const int r0 = rb + row_sub;
-      uint32_t w[R][kWords];
-      float sc[R], zc[R], v[R];
+      uint32_t w[RR][kWords];
+      float sc[RR], zc[RR], v[RR];
 #pragma unroll
-      for (int k = 0; k < R; ++k) {
+      for (int k = 0; k < RR; ++k) {
         const int rl = min(r0 + k * RS, cr - 1);
         load_unit<kWords>(cbase + rl * row_bytes, w[k], half_first);
         sc[k] = __half2float(sp[rl * G]);
         zc[k] = __half2float(zp[rl * G]);
       }
 #pragma unroll
-      for (int k = 0; k < R; ++k) {
+      for (int k = 0; k < RR; ++k) {
         const float d = unit_dot<B, kIntPath>(w[k], xr, uscale);
         v[k] = unit_ok ? sc[k] * fmaf(-zc[k], sx, d) : 0.f;
       }
-      reduce_store_rows<UW, R>(v, lane, pchunk, r0, RS, cr, NW);
+      reduce_store_rows<UW, RR>(v, lane, pchunk, r0, RS, cr, NW);
+    };
+    // Full passes while more than (R - 1) RS rows remain; a short remainder
+    // (the last rows of a CTA's share) goes RS rows at a time.  8-bit codes
+    // keep full passes (measured: the one-row pass made them slower).
+    for (int rb = 0; rb < cr;) {
+      if constexpr (B != 8) {
+        if (cr - rb <= (R - 1) * RS) {
+          pass(rb, int_<1>{});
+          rb += RS;
+          continue;
+        }
+      }
+      pass(rb, int_<R>{});
+      rb += R * RS;
     }
     if (ring) {
       __syncwarp();
