@@ -67,13 +67,18 @@ def measured_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
-def kernel_source_hash() -> str:
-    """Hash of the device/host code that builds the kernels (csrc/), so that
-    counters taken on other sources are not reported."""
+# The .cu file that defines each workload kind's dominant kernel.
+KERNEL_FILE = {"gemv": "qlin_gemv.cu", "stack": "qlin_gemv.cu", "gemm": "qlin_gemm.cu"}
+
+
+def kernel_source_hash(kind: str = None) -> str:
+    """Hash of the sources of a workload kind's dominant kernel (its .cu file
+    and the headers every kernel file includes), or of all of csrc/ when kind
+    is None, so that counters taken on other sources are not reported."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dequant_gemv_packed_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
+        if f.endswith((".cuh", ".h")) or (f.endswith(".cu") and (kind is None or f == KERNEL_FILE[kind])):
             h.update(f.encode())
             h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
@@ -449,7 +454,7 @@ def run_ours(args):
     peaks = measured_peaks()
     value = whole_job_gbs(case.bytes, args.steps, world, ms)
     per_gpu_gbs = case.bytes / (ms_step * 1e-3) / 1e9
-    khash = kernel_source_hash()
+    khash = kernel_source_hash(case.kind)
     if case.kind == "gemm":
         achieved = case.flops / (ms_step * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
