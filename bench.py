@@ -56,6 +56,11 @@ WORKLOADS = {
 }
 
 
+# Default timed steps per workload kind: about a second of timed work (a
+# gate/up call is ~5 us, a stack step ~2 ms, a prefill GEMM 40-150 us).
+DEFAULT_STEPS = {"gemv": 100000, "stack": 500, "gemm": 10000}
+
+
 # --------------------------------------------------------------------------- utils
 
 def measured_peaks():
@@ -552,7 +557,8 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: about a second of timed work for the workload; 20 for --impl reference)")
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--workload", default="gateup", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -564,6 +570,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.steps is None:
+        args.steps = 20 if args.impl == "reference" else DEFAULT_STEPS[WORKLOADS[args.workload][1]]
+    if args.steps < 1:
+        ap.error("--steps must be >= 1")
     if args.impl == "reference":
         run_reference(args)
     else:
