@@ -47,6 +47,8 @@ WORKLOADS = {
     "down16": ("decode down-proj GEMV: M=16, K=9728, N=2560, int3 g128, block-128 RHT", "gemv",
                dict(fn="down", M=16)),
     "stack": ("36-layer int6 g128 decoder linear stack + int8 lm_head, M=1 (253 GEMVs per step)", "stack", {}),
+    "stack_fused": ("the same 36-layer int6 stack + int8 lm_head with q/k/v (2560->6144) and gate/up "
+                    "(2560->19456) fused, each sharing one x, M=1 (145 GEMVs per step)", "stack", dict(fused=True)),
     "prefill256": ("prefill dequant-GEMM: M=256, K=2560, N=9728, mixed int6/int8 64-row blocks, block-128 RHT",
                    "gemm", dict(M=256)),
     "prefill1024": ("prefill dequant-GEMM: M=1024, K=2560, N=9728, mixed int6/int8 64-row blocks, block-128 RHT",
@@ -214,7 +216,7 @@ class Case:
             self.layers = []
             self.bytes = 0
             self.flops = 0
-            for _, w, a in W.stack(device=dev):
+            for _, w, a in (W.stack_fused if p.get("fused") else W.stack)(device=dev):
                 d = Q.Desc.of(w)
                 packed = Q.qlin_pack(d, w.codes)
                 del w.codes

@@ -205,3 +205,36 @@ def stack(device="cpu", seed: int = 0) -> Iterator[tuple[str, QuantWeight, Activ
         w = draw_weight(N, K, bits, seed=seed, index=i + 1, device=device)
         a = draw_activation(1, K, seed=seed, index=i + 1, device=device)
         yield name, w, a
+
+
+def concat_rows(ws: list[QuantWeight]) -> QuantWeight:
+    """One weight whose output rows are those of `ws` in order (same K, same
+    uniform width): the fused projection of linears that read the same x."""
+    K, bits = ws[0].K, ws[0].bits
+    assert bits and all(w.K == K and w.bits == bits for w in ws), "fusion needs one K and one uniform width"
+    return QuantWeight(sum(w.N for w in ws), K, bits, None, torch.cat([w.codes for w in ws]),
+                       torch.cat([w.scales for w in ws]), torch.cat([w.zeros for w in ws]))
+
+
+# Projections of one layer that read the same x, fused into one weight each.
+STACK_FUSED = (("qkv_proj", ("q_proj", "k_proj", "v_proj")), ("o_proj", ("o_proj",)),
+               ("gate_up_proj", ("gate_proj", "up_proj")), ("down_proj", ("down_proj",)))
+
+
+def stack_fused(device="cpu", seed: int = 0) -> Iterator[tuple[str, QuantWeight, Activation]]:
+    """The stack's weights (the same draws as `stack`) with q/k/v and gate/up
+    each fused into one weight of N = 6144 and 19456 rows; a fused projection
+    reads the x of its first member.  Yields (name, weight, activation) for
+    the 36 x 4 fused linears and the lm_head."""
+    lin = stack_linears()
+    index = {name: i for i, (name, _, _, _) in enumerate(lin)}
+    for layer in range(STACK_LAYERS):
+        for fused, members in STACK_FUSED:
+            ids = [index[f"layers.{layer}.{m}"] for m in members]
+            ws = [draw_weight(lin[i][2], lin[i][1], lin[i][3], seed=seed, index=i + 1, device=device) for i in ids]
+            a = draw_activation(1, lin[ids[0]][1], seed=seed, index=ids[0] + 1, device=device)
+            yield f"layers.{layer}.{fused}", (ws[0] if len(ws) == 1 else concat_rows(ws)), a
+    i = len(lin) - 1
+    name, K, N, bits = lin[i]
+    yield name, draw_weight(N, K, bits, seed=seed, index=i + 1, device=device), \
+        draw_activation(1, K, seed=seed, index=i + 1, device=device)

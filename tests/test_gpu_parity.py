@@ -155,6 +155,32 @@ def test_gemv_stack_int6_int8_sampled():
     print("stack worst rel errors", worst)
 
 
+def test_gemv_fused_projections():
+    """Fused q/k/v (N = 6144) and gate/up (N = 19456) of one layer: one weight of
+    the members' rows and one x.  Sampled rows of every member against the
+    oracle; all rows consistent with the members' separate calls."""
+    lin = W.stack_linears()
+    index = {name: i for i, (name, _, _, _) in enumerate(lin)}
+    for members in (("q_proj", "k_proj", "v_proj"), ("gate_proj", "up_proj")):
+        ids = [index[f"layers.0.{m}"] for m in members]
+        ws = [W.draw_weight(lin[i][2], lin[i][1], lin[i][3], seed=0, index=i + 1, device=DEV) for i in ids]
+        a = W.draw_activation(1, lin[ids[0]][1], seed=0, index=ids[0] + 1, device=DEV)
+        f = W.concat_rows(ws)
+        rows, r0 = [], 0
+        for k, w in enumerate(ws):  # both ends of every member's row range
+            rows.extend((r0 + sample_rows(w.N, 16, seed=k)).tolist())
+            r0 += w.N
+        _gemv_case(f, a, rows, what="+".join(members))
+        d, packed = packed_on_device(f)
+        y = Q.qlin_gemv(d, packed, f.scales, f.zeros, a.sign_bits, a.x)
+        parts = []
+        for w in ws:
+            dw, pw = packed_on_device(w)
+            parts.append(Q.qlin_gemv(dw, pw, w.scales, w.zeros, a.sign_bits, a.x))
+        separate = torch.cat(parts, dim=1).double().cpu().numpy()
+        assert_close(y, separate, what="+".join(members) + " fused vs separate calls")
+
+
 @pytest.mark.parametrize("bits", [3, 4, 6, 8])
 @pytest.mark.parametrize("N,K,M", [(1, 128, 1), (77, 384, 5), (333, 1280, 16), (64, 9728, 2)])
 def test_gemv_ragged(bits, N, K, M):

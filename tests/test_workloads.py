@@ -58,3 +58,30 @@ def test_stack_shapes():
     assert lin[-1] == ("lm_head", 2560, 151936, 8)
     total_weights = sum(K * N for _, K, N, _ in lin)
     assert total_weights == 36 * (2560 * 4096 + 2 * 2560 * 1024 + 4096 * 2560 + 2 * 2560 * 9728 + 9728 * 2560) + 2560 * 151936
+
+
+def test_concat_rows():
+    ws = [W.draw_weight(n, 256, 4, seed=0, index=i + 1) for i, n in enumerate((64, 3, 128))]
+    f = W.concat_rows(ws)
+    assert (f.N, f.K, f.bits) == (195, 256, 4)
+    assert torch.equal(f.codes[64:67], ws[1].codes) and torch.equal(f.scales[67:], ws[2].scales)
+    assert torch.equal(f.zeros[:64], ws[0].zeros)
+    try:
+        W.concat_rows([ws[0], W.draw_weight(8, 128, 4, seed=0)])
+    except AssertionError:
+        pass
+    else:
+        raise AssertionError("rows of different K were fused")
+
+
+def test_stack_fused_first_projection():
+    """The fused q/k/v of layer 0 is the stack's q, k and v rows in order and
+    reads the x of q."""
+    import itertools
+    name, f, a = next(W.stack_fused())
+    sep = list(itertools.islice(W.stack(), 3))
+    assert name == "layers.0.qkv_proj" and f.N == 6144 and f.K == 2560 and f.bits == 6
+    assert torch.equal(f.codes, torch.cat([w.codes for _, w, _ in sep]))
+    assert torch.equal(f.scales, torch.cat([w.scales for _, w, _ in sep]))
+    assert torch.equal(a.x, sep[0][2].x) and torch.equal(a.sign_bits, sep[0][2].sign_bits)
+    assert [n for n, _ in W.STACK_FUSED] == ["qkv_proj", "o_proj", "gate_up_proj", "down_proj"]
