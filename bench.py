@@ -49,6 +49,8 @@ WORKLOADS = {
     "stack": ("36-layer int6 g128 decoder linear stack + int8 lm_head, M=1 (253 GEMVs per step)", "stack", {}),
     "stack_fused": ("the same 36-layer int6 stack + int8 lm_head with q/k/v (2560->6144) and gate/up "
                     "(2560->19456) fused, each sharing one x, M=1 (145 GEMVs per step)", "stack", dict(fused=True)),
+    "quantize": ("offline weight side: rotation (signs + block-128 FWHT, fp64) and RTN int4 g128 quantisation "
+                 "of an fp16 weight, K=2560, N=9728", "quantize", dict(N=9728, K=2560, bits=4)),
     "prefill256": ("prefill dequant-GEMM: M=256, K=2560, N=9728, mixed int6/int8 64-row blocks, block-128 RHT",
                    "gemm", dict(M=256)),
     "prefill1024": ("prefill dequant-GEMM: M=1024, K=2560, N=9728, mixed int6/int8 64-row blocks, block-128 RHT",
@@ -60,7 +62,7 @@ WORKLOADS = {
 
 # Default timed steps per workload kind: about a second of timed work (a
 # gate/up call is ~5 us, a stack step ~2 ms, a prefill GEMM 40-150 us).
-DEFAULT_STEPS = {"gemv": 100000, "stack": 500, "gemm": 10000}
+DEFAULT_STEPS = {"gemv": 100000, "stack": 500, "gemm": 10000, "quantize": 20000}
 
 
 # --------------------------------------------------------------------------- utils
@@ -75,7 +77,8 @@ def measured_peaks():
 
 
 # The .cu file that defines each workload kind's dominant kernel.
-KERNEL_FILE = {"gemv": "qlin_gemv.cu", "stack": "qlin_gemv.cu", "gemm": "qlin_gemm.cu"}
+KERNEL_FILE = {"gemv": "qlin_gemv.cu", "stack": "qlin_gemv.cu", "gemm": "qlin_gemm.cu", "quantize": "qlin_quant.cu"}
+QUANTIZE_METRIC = "µs/call and achieved HBM GB/s (fraction of ~8 TB/s) of the offline weight rotation + RTN quantisation"
 
 
 def kernel_source_hash(kind: str = None) -> str:
@@ -230,6 +233,27 @@ class Case:
             self.host_sample = None
             torch.cuda.synchronize()
             return
+        if kind == "quantize":
+            N, K, bits = p["N"], p["K"], p["bits"]
+            self.M, self.N, self.K, self.bits, self.block_bits = 1, N, K, bits, None
+            self.d = Q.Desc(N, K, bits)
+            w = W.draw_fp16_weight(N, K, device=dev)
+            a = W.draw_activation(1, K, device=dev)
+            G = K // 128
+            # algorithmic bytes: read the fp16 weight, write codes (one byte each) and fp16 scale/zero
+            self.bytes = N * K * 2 + N * K + 4 * N * G
+            self.flops = 0
+            self.copies = copies or max(1, math.ceil(2 * L2_BYTES / (N * K * 2)) + 1)
+            self.w = [w.clone() for _ in range(self.copies)]
+            self.out = [(torch.empty(N, K, dtype=torch.uint8, device=dev),
+                         torch.empty(N, G, dtype=torch.float16, device=dev),
+                         torch.empty(N, G, dtype=torch.float16, device=dev)) for _ in range(2)]
+            self.weight_bytes_total = self.copies * N * K * 2
+            self.sign_bits, self.x = a.sign_bits, a.x
+            self.host_sample = (w.cpu().numpy(), a.sign_bits.cpu().numpy().view(np.uint32))
+            del w
+            torch.cuda.synchronize()
+            return
         if kind == "gemv":
             fn = getattr(W, p["fn"])
             w, a = fn(device=dev, M=p["M"]) if p["fn"] != "tiny" else fn(device=dev)
@@ -261,12 +285,18 @@ class Case:
 
     def launches_per_step(self) -> int:
         from dequant_gemv_packed_b200 import qlin as Q
+        if self.kind == "quantize":
+            return 1  # uniform width: one launch
         if self.kind == "stack":
             return sum(Q.kernel_launches_per_call("gemv", l[0], 1) for l in self.layers)
         return Q.kernel_launches_per_call(self.kind, self.d, self.M)
 
     def step(self, i: int):
         Q = self.Q
+        if self.kind == "quantize":
+            c, sc, z = self.out[i % 2]
+            Q.qlin_quantize_rtn(self.d, self.w[i % self.copies], self.sign_bits, c, sc, z)
+            return
         if self.kind == "stack":
             for (d, packed, s, z, sb, x, y, ws) in self.layers:
                 Q.qlin_gemv(d, packed, s, z, sb, x, y, ws)
@@ -328,6 +358,8 @@ def time_e2e(case: Case, K: int, W: int, stream):
     memory, run the layer, copy y back to pinned host memory."""
     if case.kind == "stack":
         return None
+    if case.kind == "quantize":
+        return time_e2e_quantize(case, K, W, stream)
     n = min(K, 2000)
     xh = case.x.cpu().pin_memory()
     yh = torch.empty(case.M, case.N, dtype=torch.float16).pin_memory()
@@ -354,9 +386,41 @@ def time_e2e(case: Case, K: int, W: int, stream):
             "steps": n, "mode": "eager calls through the Python binding"}
 
 
+def time_e2e_quantize(case: Case, K: int, W: int, stream):
+    """The offline tool through the public binding, eager: per step copy the fp16
+    weight in from pinned host memory, quantise, copy codes, scales and zeros
+    back to pinned host memory."""
+    n = min(K, 200)
+    wh = case.w[0].cpu().pin_memory()
+    c, sc, z = case.out[0]
+    ch, sh, zh = c.cpu().pin_memory(), sc.cpu().pin_memory(), z.cpu().pin_memory()
+    wd = torch.empty_like(case.w[0])
+    Q = case.Q
+    with torch.cuda.stream(stream):
+        def one():
+            wd.copy_(wh, non_blocking=True)
+            Q.qlin_quantize_rtn(case.d, wd, case.sign_bits, c, sc, z)
+            ch.copy_(c, non_blocking=True)
+            sh.copy_(sc, non_blocking=True)
+            zh.copy_(z, non_blocking=True)
+        for _ in range(min(W, 10)):
+            one()
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(n):
+            one()
+        end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / n
+    return {"value": case.bytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "us_per_call": ms * 1e3,
+            "h2d_bytes_per_step": wh.numel() * 2, "d2h_bytes_per_step": ch.numel() + 2 * sh.numel() * 2,
+            "steps": n, "mode": "eager calls through the Python binding"}
+
+
 def time_cublas(case: Case, stream, reps: int = 2000):
     """bf16 torch.nn.functional.linear (cuBLAS) of the same shape, same rotation."""
-    if case.kind == "stack":
+    if case.kind in ("stack", "quantize"):
         return None
     copies = max(1, math.ceil(2 * L2_BYTES / (case.N * case.K * 2)) + 1)
     ws = [torch.randn(case.N, case.K, device="cuda", dtype=torch.bfloat16) for _ in range(copies)]
@@ -402,6 +466,26 @@ def case_host_packed(case_host, bits, block_bits):
         from oracle import qlin_oracle as O
         _PACKED_CACHE[key] = O.pack(case_host[0], bits or None, None if bits else block_bits)
     return _PACKED_CACHE[key]
+
+
+def cpu_quantize_rate(case: Case, budget_s: float = 12.0):
+    """Oracle throughput of the offline tool (GB/s of its algorithmic bytes) on
+    row samples of the weight, BLAS limited to one thread."""
+    from threadpoolctl import threadpool_limits
+    from oracle import qlin_oracle as O
+    w, sb = case.host_sample
+    N = w.shape[0]
+    per_row = case.bytes / N
+    rng = np.random.default_rng(0)
+    done_rows, t = 0, 0.0
+    with threadpool_limits(limits=1):
+        while t < budget_s and done_rows < N:
+            rows = np.sort(rng.choice(N, size=min(256, N), replace=False))
+            t1 = time.perf_counter()
+            O.quantize_rtn(w[rows], sb, case.bits)
+            t += time.perf_counter() - t1
+            done_rows += len(rows)
+    return done_rows * per_row / t / 1e9, done_rows, t
 
 
 def cpu_oracle_rate(case: Case, budget_s: float = 12.0, rows_per_step: int | None = None):
@@ -477,23 +561,29 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and case.host_sample is not None and not args.no_cpu_baseline \
             and not args.no_extras:
-        gbs, rows, t = cpu_oracle_rate(case, budget_s=args.cpu_budget)
+        if case.kind == "quantize":
+            gbs, rows, t = cpu_quantize_rate(case, budget_s=args.cpu_budget)
+            what = "explicit-H fp64 rotation + fp32 RTN"
+        else:
+            gbs, rows, t = cpu_oracle_rate(case, budget_s=args.cpu_budget)
+            what = "unpack + fp64 dequant + explicit-H rotation + fp64 matmul"
         cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"{rows} of {case.N} weight rows (unpack + fp64 dequant + explicit-H rotation + fp64 "
-                         f"matmul), {t:.1f} s, BLAS limited to 1 thread"}
+               "sample": f"{rows} of {case.N} weight rows ({what}), {t:.1f} s, BLAS limited to 1 thread"}
     if rank == 0:
         us = ms_step * 1e3
         cfg = {"workload": case.desc_text, "M": case.M, "K": case.K, "N": case.N,
                "group": 128, "copies": case.copies,
                "l2": f"rotating {case.copies} weight copies ({case.weight_bytes_total / 1e6:.0f} MB > 2x L2)"
                if case.kind != "stack" else f"stack weights {case.weight_bytes_total / 1e9:.2f} GB > L2",
-               "parallelism": f"replicas x{world}", "accumulate": "fp32", "kernel_hash": khash,
+               "parallelism": f"replicas x{world}",
+               "accumulate": "fp64 rotation, fp32 quantiser" if case.kind == "quantize" else "fp32",
+               "kernel_hash": khash,
                "launch": ("CUDA graph, consecutive calls overlapped by programmatic dependent launch "
                           "(qlin_set_overlap(1))") if overlap else "CUDA graph, serial launches"}
-        out = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        out = {"metric": QUANTIZE_METRIC if case.kind == "quantize" else METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
                "warmup": args.warmup, "ms_per_step": ms_step, "us_per_call": us,
-               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-               "data": "synthetic", "config": cfg, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+               "dtype": "f64" if case.kind == "quantize" else "f16", "data": "synthetic", "config": cfg, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                "gpu_launches": case.launches_per_step() * args.steps, "clocks": clocks}
         if cublas_us is not None:
             out["cublas_bf16"] = {"us_per_call": cublas_us, "speedup": cublas_us / us}
@@ -515,6 +605,9 @@ def run_reference(args):
     desc, kind, p = WORKLOADS[args.workload]
     if kind == "stack":
         print(json.dumps({"impl": "reference", "unavailable": "stack workload is not sampled by the CPU oracle arm"}))
+        return
+    if kind == "quantize":
+        run_reference_quantize(args, desc, p)
         return
     if kind == "gemv":
         fn = getattr(W, p["fn"])
@@ -551,6 +644,41 @@ def run_reference(args):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": {"workload": desc, "M": a.x.shape[0], "K": K, "N": N, "group": 128},
+           "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def run_reference_quantize(args, desc, p):
+    """Reference arm of the offline tool: the oracle on sampled rows per step."""
+    from dequant_gemv_packed_b200 import workloads as W
+    from oracle import qlin_oracle as O
+    from threadpoolctl import threadpool_limits
+    N, K, bits = p["N"], p["K"], p["bits"]
+    w = W.draw_fp16_weight(N, K).numpy()
+    sb = W.draw_activation(1, K).sign_bits.numpy().view(np.uint32)
+    per_row = (N * K * 3 + 4 * N * (K // 128)) / N
+    rng = np.random.default_rng(0)
+    total_budget = float(os.environ.get("QLIN_REFERENCE_BUDGET_S", "90"))
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        O.quantize_rtn(w[:64], sb, bits)
+        t_row = (time.perf_counter() - t0) / 64
+        rows_per_step = int(max(4, min(N, total_budget / max(args.steps + args.warmup, 1) / t_row)))
+        def step():
+            O.quantize_rtn(w[np.sort(rng.choice(N, size=rows_per_step, replace=False))], sb, bits)
+        for _ in range(args.warmup):
+            step()
+        t1 = time.perf_counter()
+        for _ in range(args.steps):
+            step()
+        t = time.perf_counter() - t1
+    value = rows_per_step * per_row * args.steps / t / 1e9
+    sample = f"{rows_per_step} of {N} weight rows per step (explicit-H fp64 rotation + fp32 RTN)"
+    out = {"impl": "reference", "metric": QUANTIZE_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3 / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": desc, "K": K, "N": N, "group": 128, "bits": bits},
            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)

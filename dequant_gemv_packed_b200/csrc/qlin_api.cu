@@ -150,6 +150,18 @@ qlin_status qlin_dequant(const qlin_desc* d, const void* packed, const uint16_t*
                         reinterpret_cast<cudaStream_t>(st));
 }
 
+qlin_status qlin_quantize_rtn(const qlin_desc* d, const uint16_t* w, const uint32_t* sign_bits, uint8_t* codes,
+                              uint16_t* scales, uint16_t* zeros, qlin_stream_t st) {
+  qlin_status r = check_desc(d);
+  if (r != QLIN_OK) return r;
+  if (!w || !sign_bits || !codes || !scales || !zeros) return QLIN_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(sign_bits) || !aligned16(codes) || !aligned16(scales) || !aligned16(zeros))
+    return QLIN_ERR_ALIGNMENT;
+  return launch_quantize_rtn(reinterpret_cast<const __half*>(w), sign_bits, d->block_bits, d->bits, d->N, d->K,
+                             codes, reinterpret_cast<__half*>(scales), reinterpret_cast<__half*>(zeros),
+                             reinterpret_cast<cudaStream_t>(st));
+}
+
 qlin_status qlin_rht(const uint16_t* x, uint16_t* xr, const uint32_t* sign_bits, int32_t M,
                      int32_t K, qlin_stream_t st) {
   if (!x || !xr || !sign_bits) return QLIN_ERR_INVALID_ARG;

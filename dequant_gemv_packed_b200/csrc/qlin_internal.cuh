@@ -53,6 +53,9 @@ unsigned take_gemm_error();
 qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half* zeros,
                         const uint32_t* sign_bits, const __half* x, __half* y, int M,
                         void* workspace, cudaStream_t s);
+// Rotation and round-to-nearest quantisation of fp16 weight rows (offline tool).
+qlin_status launch_quantize_rtn(const __half* w, const uint32_t* sign_bits, const uint8_t* block_bits, int bits,
+                                int N, int K, uint8_t* codes, __half* scales, __half* zeros, cudaStream_t s);
 size_t gemm_workspace_bytes(int M, int K);
 qlin_status launch_gemm(const PackedView& v, const __half* scales, const __half* zeros,
                         const uint32_t* sign_bits, const __half* x, __half* y, int M,

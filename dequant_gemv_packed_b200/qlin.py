@@ -23,6 +23,7 @@ EXPORTED = (
     "qlin_status_string", "qlin_last_cuda_error", "qlin_packed_bytes", "qlin_code_bytes", "qlin_pack",
     "qlin_unpack", "qlin_dequant", "qlin_rht", "qlin_gemv_workspace_bytes", "qlin_gemv",
     "qlin_gemm_workspace_bytes", "qlin_gemm", "qlin_device_error", "qlin_gemm_noalloc", "qlin_set_overlap",
+    "qlin_quantize_rtn",
 )
 
 
@@ -83,6 +84,7 @@ def lib() -> ctypes.CDLL:
     L.qlin_unpack.argtypes, L.qlin_unpack.restype = [vp, vp, vp, vp], ctypes.c_int
     L.qlin_dequant.argtypes, L.qlin_dequant.restype = [vp, vp, vp, vp, vp, vp], ctypes.c_int
     L.qlin_rht.argtypes, L.qlin_rht.restype = [vp, vp, vp, i32, i32, vp], ctypes.c_int
+    L.qlin_quantize_rtn.argtypes, L.qlin_quantize_rtn.restype = [vp, vp, vp, vp, vp, vp, vp], ctypes.c_int
     L.qlin_gemv_workspace_bytes.argtypes, L.qlin_gemv_workspace_bytes.restype = [vp, i32], sz
     L.qlin_gemm_workspace_bytes.argtypes, L.qlin_gemm_workspace_bytes.restype = [vp, i32], sz
     L.qlin_device_error.argtypes, L.qlin_device_error.restype = [ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int
@@ -186,6 +188,22 @@ def qlin_dequant(desc: Desc, packed: torch.Tensor, scales: torch.Tensor, zeros: 
                               _dev(zeros, torch.float16, "zeros"), _dev(w, torch.float16, "w"), _stream(stream)),
            "qlin_dequant")
     return w
+
+
+def qlin_quantize_rtn(desc: Desc, w: torch.Tensor, sign_bits: torch.Tensor, codes: Optional[torch.Tensor] = None,
+                      scales: Optional[torch.Tensor] = None, zeros: Optional[torch.Tensor] = None, stream=None):
+    """Rotated round-to-nearest quantisation of fp16 weight rows: (codes, scales, zeros)."""
+    G = desc.K // 128
+    if codes is None:
+        codes = _alloc((desc.N, desc.K), torch.uint8, w)
+    if scales is None:
+        scales = _alloc((desc.N, G), torch.float16, w)
+    if zeros is None:
+        zeros = _alloc((desc.N, G), torch.float16, w)
+    _check(lib().qlin_quantize_rtn(desc.ref(), _dev(w, torch.float16, "w"), _dev(sign_bits, torch.int32, "sign_bits"),
+                                   _dev(codes, torch.uint8, "codes"), _dev(scales, torch.float16, "scales"),
+                                   _dev(zeros, torch.float16, "zeros"), _stream(stream)), "qlin_quantize_rtn")
+    return codes, scales, zeros
 
 
 def qlin_rht(x: torch.Tensor, sign_bits: torch.Tensor, xr: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

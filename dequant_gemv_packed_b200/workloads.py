@@ -96,10 +96,9 @@ def rtn_quantise(w: torch.Tensor, bits: int) -> tuple[torch.Tensor, torch.Tensor
     return q.to(torch.uint8).reshape(N, K), s16, z16
 
 
-def draw_weight(N: int, K: int, bits: int, *, seed: int = 0, index: int = 0, outliers: bool = True,
-                block_bits: Optional[torch.Tensor] = None, device="cpu") -> QuantWeight:
-    """Draw W ~ N(0, 0.02) [N, K] (fp32), scale exactly round(0.1 % * N * K) entries,
-    chosen without replacement, by 20, and RTN-quantise each row with its width."""
+def _draw_w32(N: int, K: int, seed: int, index: int, outliers: bool, device) -> torch.Tensor:
+    """W ~ N(0, 0.02) [N, K] (fp32) with exactly round(0.1 % * N * K) entries,
+    chosen without replacement, scaled by 20."""
     gw = _gen(device, seed, _STREAM_WEIGHTS, index)
     w = torch.randn(N, K, generator=gw, device=device, dtype=torch.float32) * WEIGHT_STD
     if outliers:
@@ -108,6 +107,21 @@ def draw_weight(N: int, K: int, bits: int, *, seed: int = 0, index: int = 0, out
         pos = torch.randperm(N * K, generator=go, device=device)[:n_out]
         w.view(-1)[pos] *= OUTLIER_FACTOR
         del pos
+    return w
+
+
+def draw_fp16_weight(N: int, K: int, *, seed: int = 0, index: int = 0, outliers: bool = True,
+                     device="cpu") -> torch.Tensor:
+    """The unquantised weight of `draw_weight` (same draw), rounded to fp16: the
+    input of the offline rotation and quantisation."""
+    return _draw_w32(N, K, seed, index, outliers, device).half()
+
+
+def draw_weight(N: int, K: int, bits: int, *, seed: int = 0, index: int = 0, outliers: bool = True,
+                block_bits: Optional[torch.Tensor] = None, device="cpu") -> QuantWeight:
+    """Draw W ~ N(0, 0.02) [N, K] (fp32), scale exactly round(0.1 % * N * K) entries,
+    chosen without replacement, by 20, and RTN-quantise each row with its width."""
+    w = _draw_w32(N, K, seed, index, outliers, device)
     if bits:
         codes, s, z = rtn_quantise(w, bits)
         return QuantWeight(N, K, bits, None, codes, s, z)

@@ -150,6 +150,32 @@ qlin_status qlin_unpack(const qlin_desc* desc, const void* packed, uint8_t* code
 qlin_status qlin_dequant(const qlin_desc* desc, const void* packed, const uint16_t* scales,
                          const uint16_t* zeros, uint16_t* w, qlin_stream_t stream);
 
+/* Offline weight side: rotate each weight row along K with the activations'
+ * signs and block-128 Hadamard, then quantise it by asymmetric round-to-nearest
+ * per group of 128, ready for qlin_pack with the same descriptor:
+ *   w~ = fp32( fp64(1/sqrt(128)) * (H_128 diag(d) w) )   per block of 128
+ *        (the sum exact in fp64, one multiply, sqrt and division rounded to
+ *        nearest, then one rounding to fp32),
+ *   s  = fp16_rn( (max w~ - min w~) / (2^b - 1) ), replaced by 1 if not > 0,
+ *   z  = fp16_rn( -min w~ / s ),
+ *   q  = min(max(rint(w~ / s + z), 0), 2^b - 1)
+ * with every fp32 operation rounded to nearest and nothing fused, so the
+ * outputs are a function of the input alone (bit-exact, deterministic).  A zero
+ * minimum counts as +0 (z is then -0).  Inputs beyond the fp16 range of s are
+ * not guarded.
+ *   w        : device fp16 [N][K], the unrotated weight;
+ *   sign_bits: device uint32 [K/32] (bit k set: d_k = -1), the signs qlin_gemv
+ *              applies to x;
+ *   codes    : device uint8 [N][K];  scales, zeros : device fp16 [N][K/128].
+ * Widths: desc->bits, or per 64-row block from desc->block_bits (one launch per
+ * run of equal widths).  No buffer may alias another.
+ * Definition: "24B0978-Week01-Track2_20-Submission01", paragraph "Random
+ * Hadamard transform" (the weight side is rotated offline, before
+ * quantisation); "24B0978-Week02-Track2-40-Submission01", recipe op
+ * "quant_rtn" (bits, group 128). */
+qlin_status qlin_quantize_rtn(const qlin_desc* desc, const uint16_t* w, const uint32_t* sign_bits,
+                              uint8_t* codes, uint16_t* scales, uint16_t* zeros, qlin_stream_t stream);
+
 /* Random Hadamard transform of M rows of K activations.
  *   x  : device fp16 [M][K];  xr : device fp16 [M][K] (may not alias x);
  *   sign_bits : device uint32 [K/32].

@@ -26,6 +26,14 @@ What it computes, in the plainest form that the pages support
   Dense 128x128 products, not a butterfly.
 * ``linear64`` -- the fp64 matmul of the rotated activations with the fp64
   dequantised weight.
+* ``rotate_weight32`` / ``rtn32`` / ``quantize_rtn`` -- the offline weight side:
+  each weight row rotated with the activations' signs and H / sqrt(128) (the
+  weight side of the rotation is folded in offline, "24B0978-Week01-Track2_20-
+  Submission01", paragraph "Random Hadamard transform"), rounded once to fp32,
+  then asymmetric round-to-nearest per group of 128 ("24B0978-Week02-Track2-40-
+  Submission01", recipe op "quant_rtn": bits, group 128) in fp32 arithmetic:
+  s = fp16((max - min) / (2^b - 1)) (1 if not > 0), z = fp16(-min / s),
+  q = clip(rint(w / s + z), 0, 2^b - 1).
 
 Readings where the pages leave a step open (the library documents the same readings):
 
@@ -35,6 +43,8 @@ Readings where the pages leave a step open (the library documents the same readi
   before H.
 * The rotated activation is rounded once to fp16 (``rht16``).
 * Code bits above the width are ignored by ``pack``.
+* Round-to-nearest quantisation works per group in fp32 with the min/max
+  affine form above; a zero minimum counts as +0 (so z is -0).
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 against closed forms, brute force, exact rational arithmetic or a library
@@ -201,6 +211,45 @@ def rht64(x: np.ndarray, sign_bits: np.ndarray) -> np.ndarray:
 def rht16(x: np.ndarray, sign_bits: np.ndarray) -> np.ndarray:
     """The rotated activation rounded once to fp16."""
     return rht64(x, sign_bits).astype(np.float16)
+
+
+# --------------------------------------------------------------------------
+# Offline weight side: rotation and round-to-nearest quantisation
+# --------------------------------------------------------------------------
+
+def rotate_weight32(w: np.ndarray, sign_bits: np.ndarray) -> np.ndarray:
+    """Each fp16 weight row rotated like the activations (``rht64``: signs, then
+    H / sqrt(128) per block of 128), rounded once to fp32.  For fp16 input the
+    fp64 sums are exact (multiples of 2^-24 below 2^23), so this is the fp32
+    rounding of one fp64 product of the exact sum with 1/sqrt(128)."""
+    return rht64(np.asarray(w, np.float16).astype(np.float64), sign_bits).astype(np.float32)
+
+
+def rtn32(wr: np.ndarray, bits: int | None = None, block_bits=None):
+    """Asymmetric round-to-nearest per group of 128 of fp32 rows ``wr`` [N, K],
+    every step an fp32 operation rounded to nearest:
+    s = fp16((max - min) / (2^b - 1)), replaced by 1 unless > 0;
+    z = fp16(-min / s) with a zero minimum taken as +0;
+    q = clip(rint(w / s + z), 0, 2^b - 1).
+    Returns (codes uint8 [N, K], scales fp16 [N, K/128], zeros fp16 [N, K/128])."""
+    wr = np.asarray(wr, np.float32)
+    N, K = wr.shape
+    g = wr.reshape(N, K // GROUP, GROUP)
+    qmax = (np.float32(2.0) ** row_widths(N, bits, block_bits).astype(np.float32) - np.float32(1.0))[:, None]
+    mn = g.min(axis=-1) + np.float32(0.0)
+    mx = g.max(axis=-1)
+    s16 = ((mx - mn) / qmax).astype(np.float16)
+    s16 = np.where(s16.astype(np.float32) > np.float32(0.0), s16, np.float16(1.0))
+    s32 = s16.astype(np.float32)
+    z16 = (-mn / s32).astype(np.float16)
+    z32 = z16.astype(np.float32)
+    q = np.clip(np.rint(g / s32[..., None] + z32[..., None]), np.float32(0.0), qmax[..., None])
+    return q.astype(np.uint8).reshape(N, K), s16, z16
+
+
+def quantize_rtn(w: np.ndarray, sign_bits: np.ndarray, bits: int | None = None, block_bits=None):
+    """The offline weight side: ``rtn32(rotate_weight32(w))``."""
+    return rtn32(rotate_weight32(w, sign_bits), bits, block_bits)
 
 
 # --------------------------------------------------------------------------

@@ -103,3 +103,18 @@ def test_library_refuses_without_build(tmp_path, monkeypatch):
     monkeypatch.setattr(Q, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         Q.lib()
+
+
+def test_quantize_validation_returns_before_launch(lib):
+    """qlin_quantize_rtn rejects null, misaligned and bad-shape arguments
+    before any CUDA call (the pointers here are never dereferenced)."""
+    p = ctypes.c_void_p(16)
+    d = Q.Desc(64, 128, 4)
+    assert lib.qlin_quantize_rtn(None, p, p, p, p, p, None) == -1
+    assert lib.qlin_quantize_rtn(d.ref(), None, p, p, p, p, None) == -1
+    assert lib.qlin_quantize_rtn(d.ref(), p, p, p, p, None, None) == -1
+    assert lib.qlin_quantize_rtn(d.ref(), ctypes.c_void_p(18), p, p, p, p, None) == -4
+    assert lib.qlin_quantize_rtn(d.ref(), p, p, ctypes.c_void_p(24), p, p, None) == -4
+    assert lib.qlin_quantize_rtn(Q.Desc(64, 100, 4).ref(), p, p, p, p, p, None) == -3
+    assert lib.qlin_quantize_rtn(Q.Desc(64, 128, 5).ref(), p, p, p, p, p, None) == -2
+    assert lib.qlin_quantize_rtn(Q.Desc(65, 128, 0, [6, 6]).ref(), p, p, p, p, p, None) == -3

@@ -209,6 +209,49 @@ def test_gemv_m1_tall_shapes(bits, N, K):
     _gemv_case(w, a, what=f"b{bits} N{N} K{K} M1")
 
 
+def _quantize_case(N, K, bits, block_bits=None, seed=0):
+    w = W.draw_fp16_weight(N, K, seed=seed, index=N + K)
+    w[0, :128] = 0.0                        # a zero group (rotated: zeros of both signs)
+    w[-1, -128:] = 0.25                     # a constant group
+    if N > 2:
+        w[1, :128] = 0.0                    # a one-hot group (rotated: +-c only)
+        w[1, 5] = 0.5
+    a = W.draw_activation(1, K, seed=seed, index=N + K)
+    d = Q.Desc(N, K, bits, block_bits)
+    c, s, z = Q.qlin_quantize_rtn(d, w.to(DEV), a.sign_bits.to(DEV))
+    rc, rs, rz = O.quantize_rtn(w.numpy(), np_u32(a.sign_bits), bits or None, block_bits)
+    assert np.array_equal(c.cpu().numpy(), rc), "codes differ"
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), rs.view(np.uint16)), "scales differ"
+    assert np.array_equal(z.cpu().numpy().view(np.uint16), rz.view(np.uint16)), "zeros differ"
+    return w, a, d, c, s, z
+
+
+@pytest.mark.parametrize("N,K,bits", [(77, 384, 3), (130, 256, 4), (64, 1280, 6), (200, 2560, 8), (1, 128, 4),
+                                      (9728, 2560, 4)])
+def test_quantize_rtn_bit_exact(N, K, bits):
+    """Offline rotation + round-to-nearest on the GPU: codes, scales and zeros
+    bit-exact against the oracle (zero, constant and signed-zero groups,
+    outliers, a single row, the gate/up shape)."""
+    _quantize_case(N, K, bits)
+
+
+def test_quantize_rtn_mixed_widths_and_layer():
+    """Mixed 64-row widths (one launch per run of equal widths) bit-exact; then
+    the packed result through qlin_gemv matches the oracle layer and, the
+    rotation being folded, approximates x W^T of the unrotated weight."""
+    bb = [6, 8, 8, 4, 3, 8]
+    w, a, d, c, s, z = _quantize_case(64 * len(bb), 512, 0, bb, seed=3)
+    packed = Q.qlin_pack(d, c)
+    x = a.x.to(DEV)
+    y = Q.qlin_gemv(d, packed, s, z, a.sign_bits.to(DEV), x)
+    torch.cuda.synchronize()
+    ref = O.linear64(a.x.numpy(), c.cpu().numpy(), s.cpu().numpy(), z.cpu().numpy(), np_u32(a.sign_bits))
+    assert_close(y, ref, what="quantised layer")
+    y0 = a.x.double().numpy() @ w.double().numpy().T
+    rel = np.linalg.norm(y.double().cpu().numpy() - y0) / np.linalg.norm(y0)
+    assert rel < 0.1, rel  # RTN noise of these inputs: 0.077 (oracle), 3- and 4-bit rows dominating
+
+
 def test_gemv_mixed():
     bb = [6, 8, 4, 3, 8]
     w = _rand_weight(64 * len(bb), 1280, 0, seed=5, block_bits=bb)

@@ -362,3 +362,113 @@ def test_parity_errors():
     assert O.parity_errors(r, r) == (0.0, 0.0)
     a, f = O.parity_errors(r + np.array([[0.0, 0.0, 0.04]]), r)
     assert a == pytest.approx(0.01) and f == pytest.approx(0.04 / math.sqrt(21))
+
+
+# ------------------------------------------------- offline weight side ----
+
+def _sylvester(n):
+    """H_n by the recursion H_2n = [[H, H], [H, -H]] (integers)."""
+    h = np.array([[1]], dtype=np.int64)
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def _sign_of(sign_bits, k):
+    return -1 if (int(sign_bits[k // 32]) >> (k % 32)) & 1 else 1
+
+
+def test_rotate_weight32_exact_integer_sums():
+    """fp16 rows are integer multiples of 2^-24: the rotation as exact integer
+    sums, scaled once in fp64 by 1/sqrt(128) and rounded to fp32, equals the
+    oracle's (including subnormal and near-maximal fp16 values in one block)."""
+    rng = np.random.default_rng(11)
+    w = (rng.standard_normal((3, 256)) * 0.02).astype(np.float16)
+    w[0, :4] = [np.float16(6.0e-8), np.float16(-65504.0), np.float16(3.0e-5), np.float16(0.0)]
+    w[1, 130] = np.float16(-1.0e4)
+    sb = rng.integers(0, 2 ** 32, size=256 // 32, dtype=np.uint64).astype(np.uint32)
+    H = _sylvester(128)
+    inv = 1.0 / math.sqrt(128.0)
+    got = O.rotate_weight32(w, sb)
+    for n in range(w.shape[0]):
+        units = [int(Fraction(float(v)) * (1 << 24)) for v in w[n].astype(np.float64)]
+        for b0 in range(0, 256, 128):
+            dv = [_sign_of(sb, b0 + j) * units[b0 + j] for j in range(128)]
+            for i in range(128):
+                exact = sum(int(H[i, j]) * dv[j] for j in range(128))
+                want = np.float32(float(exact) * 2.0 ** -24 * inv)
+                assert got[n, b0 + i].view(np.uint32) == want.view(np.uint32), (n, b0, i)
+
+
+def test_rtn32_hand_cases():
+    ramp = np.tile(np.arange(16, dtype=np.float32), 8)[None, :]          # 0..15: s = 1, z = -0
+    c, s, z = O.rtn32(ramp, bits=4)
+    assert np.array_equal(c[0], ramp[0].astype(np.uint8))
+    assert s[0, 0] == np.float16(1.0) and z.view(np.uint16)[0, 0] == 0x8000
+    const = np.full((1, 128), 0.5, np.float32)                            # constant group: s = 1, z = -0.5, q = 0
+    c, s, z = O.rtn32(const, bits=6)
+    assert s[0, 0] == np.float16(1.0) and z[0, 0] == np.float16(-0.5) and not c.any()
+    zero = np.zeros((1, 128), np.float32)
+    zero[0, ::3] = -0.0                                                   # mixed zeros: still z = -0, q = 0
+    c, s, z = O.rtn32(zero, bits=3)
+    assert s[0, 0] == np.float16(1.0) and z.view(np.uint16)[0, 0] == 0x8000 and not c.any()
+    shifted = ramp + np.float32(32.0)                                     # 32..47: s = 1, z = -32
+    c, s, z = O.rtn32(shifted, bits=4)
+    assert np.array_equal(c[0], ramp[0].astype(np.uint8)) and z[0, 0] == np.float16(-32.0)
+
+
+def _ulp16(v):
+    v = abs(float(v))
+    e = max(math.floor(math.log2(v)) if v > 0 else -14, -14)
+    return Fraction(2) ** (e - 10)
+
+
+@pytest.mark.parametrize("b", [3, 4, 6, 8])
+def test_rtn32_extremes_rounding_and_error_bound(b):
+    """Against exact rationals: s is within an fp16 rounding (plus the fp32
+    quotient's) of (max - min) / (2^b - 1), z within one of -min / s; the
+    group minimum maps to 0 and maximum to 2^b - 1; every code is the nearest
+    integer to w / s + z up to the fp32 evaluation, so s (q - z) is within s/2
+    (plus that rounding) of w."""
+    rng = np.random.default_rng(b)
+    wr = (rng.standard_normal((4, 384)) * rng.uniform(0.01, 3.0, size=(4, 1))).astype(np.float32)
+    c, s, z = O.rtn32(wr, bits=b)
+    qmax = (1 << b) - 1
+    assert c.max() <= qmax
+    for n in range(4):
+        for g in range(3):
+            grp = wr[n, 128 * g:128 * (g + 1)]
+            cg = c[n, 128 * g:128 * (g + 1)]
+            mn, mx = Fraction(float(grp.min())), Fraction(float(grp.max()))
+            S, Z = Fraction(float(s[n, g])), Fraction(float(z[n, g]))
+            assert abs(S - (mx - mn) / qmax) <= _ulp16(s[n, g]) / 2 + (mx - mn) / qmax * Fraction(1, 1 << 23)
+            assert abs(Z - (-mn / S)) <= _ulp16(z[n, g]) / 2 + abs(mn / S) * Fraction(1, 1 << 23)
+            assert cg[np.argmin(grp)] == 0 and cg[np.argmax(grp)] == qmax
+            for v, q in zip(grp, cg):
+                t = Fraction(float(v)) / S + Z
+                assert abs(Fraction(int(q)) - t) <= Fraction(1, 2) + abs(t) * Fraction(1, 1 << 21), (v, q, t)
+
+
+def test_rtn32_mixed_widths():
+    rng = np.random.default_rng(5)
+    wr = rng.standard_normal((128, 256)).astype(np.float32)
+    c, _, _ = O.rtn32(wr, block_bits=[8, 3])
+    assert c[:64].max() == 255 and c[64:].max() == 7
+
+
+def test_quantize_rtn_folds_the_rotation():
+    """The weight side uses the activations' signs and H: with x rotated by
+    rht64 and W by quantize_rtn, the layer reproduces x W^T (int8: to the
+    quantisation noise)."""
+    rng = np.random.default_rng(9)
+    N, K = 40, 512
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+    x = rng.standard_normal((3, K)).astype(np.float16)
+    sb = rng.integers(0, 2 ** 32, size=K // 32, dtype=np.uint64).astype(np.uint32)
+    c, s, z = O.quantize_rtn(w, sb, bits=8)
+    y = O.linear64(x, c, s, z, sb)
+    y0 = x.astype(np.float64) @ w.astype(np.float64).T
+    rel = np.linalg.norm(y - y0) / np.linalg.norm(y0)
+    assert rel < 0.02, rel
+    bad = O.linear64(x, c, s, z, sb ^ np.uint32(1))  # one activation sign flipped: no longer the same function
+    assert np.linalg.norm(bad - y0) / np.linalg.norm(y0) > 5 * rel
