@@ -19,66 +19,83 @@
 // contraction).  The codes are a function of the input, independent of the
 // order of the butterflies.
 //
-// One warp per (row, group): lane l holds elements 4l .. 4l + 3 of the block;
-// butterfly strides 1 and 2 stay in the lane, strides 4 .. 64 are fp64
-// shuffles with lane distance 1 .. 16.
+// Eight lanes per (row, group), four groups a warp: lane t = lane % 8 of the
+// eight holds elements 16t .. 16t + 15 of the block.  Butterfly strides 1 .. 8
+// stay in the lane, strides 16, 32, 64 are fp64 shuffles with lane distance
+// 1, 2, 4; the group's min and max take three shuffle steps.
 #include "qlin_internal.cuh"
 
 namespace qlin {
 namespace {
 
 constexpr int kWarpsPerBlock = 8;
+constexpr int kGroupsPerWarp = 4;
 
 // Rows [0, N) of the arguments (already offset to the first row), all of width b.
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) quantize_rtn_kernel(
     const __half* __restrict__ w, const uint32_t* __restrict__ sign_bits, int b, int N, int K,
     uint8_t* __restrict__ codes, __half* __restrict__ scales, __half* __restrict__ zeros) {
   const int G = K / kGroup;
-  const long long item = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-  if (item >= (long long)N * G) return;  // warp-uniform
-  const int lane = threadIdx.x & 31;
-  const int n = (int)(item / G), g = (int)(item % G);
+  const long long total = (long long)N * G;
+  const int lane = threadIdx.x & 31, t = lane & 7;
+  const long long item = ((long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5)) * kGroupsPerWarp + (lane >> 3);
+  if (item - (lane >> 3) >= total) return;  // the warp's first item: warp-uniform
+  const bool live = item < total;          // lanes past the last item shuffle along on a valid one
+  const long long it = live ? item : total - 1;
+  const int n = (int)(it / G), g = (int)(it % G);
   const float qmax = (float)((1 << b) - 1);
 
-  // load 4 fp16 and their signs (bit e of the block's 128 sign bits: 1 -> -1)
-  const size_t base = (size_t)n * K + (size_t)g * kGroup + 4 * lane;
-  const uint2 raw = *reinterpret_cast<const uint2*>(w + base);
-  const uint32_t sw = sign_bits[g * 4 + (lane >> 3)] >> (4 * (lane & 7));
-  const __half2 h01 = *reinterpret_cast<const __half2*>(&raw.x);
-  const __half2 h23 = *reinterpret_cast<const __half2*>(&raw.y);
-  double v[4] = {(double)__low2float(h01), (double)__high2float(h01), (double)__low2float(h23),
-                 (double)__high2float(h23)};
+  // load 16 fp16 and their signs (bit e of the block's 128 sign bits: 1 -> -1)
+  const size_t base = (size_t)n * K + (size_t)g * kGroup + 16 * t;
+  const uint4 r0 = reinterpret_cast<const uint4*>(w + base)[0];
+  const uint4 r1 = reinterpret_cast<const uint4*>(w + base)[1];
+  const uint32_t sw = sign_bits[g * 4 + (t >> 1)] >> (16 * (t & 1));
+  const uint32_t raw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+  double v[16];
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
-    if ((sw >> j) & 1u) v[j] = -v[j];
-
-  // block FWHT (natural order), exact in fp64
-  {
-    const double a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];
-    v[0] = a0 + a2;
-    v[1] = a1 + a3;
-    v[2] = a0 - a2;
-    v[3] = a1 - a3;
+  for (int i = 0; i < 8; ++i) {
+    const __half2 h = *reinterpret_cast<const __half2*>(&raw[i]);
+    v[2 * i] = (double)__low2float(h);
+    v[2 * i + 1] = (double)__high2float(h);
   }
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const bool upper = (lane & o) != 0;
+  for (int j = 0; j < 16; ++j)
+    if ((sw >> j) & 1u) v[j] = -v[j];
+
+  // block FWHT (natural order), exact in fp64: strides 1 .. 8 in the lane
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+  for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (!(j & h)) {
+        const double u = v[j], x = v[j + h];
+        v[j] = u + x;
+        v[j + h] = u - x;
+      }
+  // strides 16, 32, 64 across the group's eight lanes
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    const bool upper = (t & o) != 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
       const double p = __shfl_xor_sync(0xffffffffu, v[j], o);
       v[j] = upper ? p - v[j] : v[j] + p;
     }
   }
   const double inv_sqrt = __ddiv_rn(1.0, __dsqrt_rn(128.0));
-  float f[4];
+  float f[16];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) f[j] = __double2float_rn(__dmul_rn(v[j], inv_sqrt));
+  for (int j = 0; j < 16; ++j) f[j] = __double2float_rn(__dmul_rn(v[j], inv_sqrt));
 
   // group minimum and maximum (exact)
-  float mn = fminf(fminf(f[0], f[1]), fminf(f[2], f[3]));
-  float mx = fmaxf(fmaxf(f[0], f[1]), fmaxf(f[2], f[3]));
+  float mn = f[0], mx = f[0];
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
+  for (int j = 1; j < 16; ++j) {
+    mn = fminf(mn, f[j]);
+    mx = fmaxf(mx, f[j]);
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   }
@@ -89,14 +106,15 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) quantize_rtn_kernel(
   const __half z16 = __float2half_rn(__fdiv_rn(-mn, s32));
   const float z32 = __half2float(z16);
 
-  uint32_t packed = 0;
+  uint32_t packed[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < 16; ++j) {
     const float q = fminf(fmaxf(rintf(__fadd_rn(__fdiv_rn(f[j], s32), z32)), 0.f), qmax);
-    packed |= (uint32_t)q << (8 * j);
+    packed[j >> 2] |= (uint32_t)q << (8 * (j & 3));
   }
-  *reinterpret_cast<uint32_t*>(codes + base) = packed;
-  if (lane == 0) {
+  if (!live) return;
+  *reinterpret_cast<uint4*>(codes + base) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  if (t == 0) {
     scales[(size_t)n * G + g] = s16;
     zeros[(size_t)n * G + g] = z16;
   }
@@ -117,7 +135,8 @@ qlin_status launch_quantize_rtn(const __half* w, const uint32_t* sign_bits, cons
       while (r1 < N && block_bits[r1 / kBlockRows] == b) r1 += kBlockRows;
     }
     const long long items = (long long)(r1 - r0) * G;
-    const long long grid = (items + kWarpsPerBlock - 1) / kWarpsPerBlock;
+    const long long per_block = (long long)kWarpsPerBlock * kGroupsPerWarp;
+    const long long grid = (items + per_block - 1) / per_block;
     if (grid > 0x7fffffffLL) return QLIN_ERR_SHAPE;
     quantize_rtn_kernel<<<(unsigned)grid, kWarpsPerBlock * 32, 0, s>>>(
         w + (size_t)r0 * K, sign_bits, b, r1 - r0, K, codes + (size_t)r0 * K, scales + (size_t)r0 * G,

@@ -309,7 +309,7 @@ def test_gemv_rejects_misaligned_and_small_workspace():
 
 # --------------------------------------------------------------- gemm ---------
 
-@pytest.mark.parametrize("M", [256, 1024, 2048])
+@pytest.mark.parametrize("M", [32, 256, 1024, 2048])
 def test_gemm_prefill_mixed_sampled(M):
     w, a = W.prefill(M=M, device=DEV)
     d, packed = packed_on_device(w)
