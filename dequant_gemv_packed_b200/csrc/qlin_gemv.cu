@@ -375,6 +375,12 @@ __device__ __forceinline__ int int4_slot(int c) {
   return 8 * (c >> 3) + 2 * (((j & 1) << 1) | (j >> 2)) + ((j >> 1) & 1);
 }
 
+// Unit u's x occupies kXw words of shared memory as 16-byte pieces; logical
+// piece i is stored at piece i ^ (u mod P), P pieces a unit, so that the lanes
+// of a load phase, which read the same piece of different units, hit distinct
+// banks.  x_half maps a 16-bit position of the unit to its place.
+__device__ __forceinline__ int x_half(int p, int u, int P) { return (((p >> 3) ^ (u & (P - 1))) << 3) | (p & 7); }
+
 // Sign flip, block-128 FWHT, x 1/sqrt(128) and fp16 rounding of one block,
 // then the unit preparation described at the top of the file.
 // The order-128 Sylvester matrix is H16 (x) H8 (element e = i + 16 j: bits
@@ -437,7 +443,7 @@ __device__ __forceinline__ void rotate_prepare(uint32_t b0, uint32_t b1, uint32_
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int c = (B == 4) ? g + 32 * (t & 1) + kOff[i] : g + kOff[i];  // position in the unit
-        xu[B == 4 ? int4_slot(c) : c] = (uint16_t)vi[i];
+        xu[x_half(B == 4 ? int4_slot(c) : c, u, kXw / 4)] = (uint16_t)vi[i];
       }
       if (leader) ust[u] = make_float2(xinv, (float)isum * xinv);
     }
@@ -452,9 +458,9 @@ __device__ __forceinline__ void rotate_prepare(uint32_t b0, uint32_t b1, uint32_
       sx += __shfl_xor_sync(0xffffffffu, sx, o);
     }
     if (store) {
-      __half* xh = reinterpret_cast<__half*>(xs) + (size_t)blk * kHadamard + g + 32 * t;
+      __half* xh = reinterpret_cast<__half*>(xu);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) xh[kOff[i]] = hv[i];
+      for (int i = 0; i < 4; ++i) xh[x_half(g + 32 * (t & 1) + kOff[i], u, kXw / 4)] = hv[i];
       if (leader) ust[u] = make_float2(corr, sx);
     }
   }
@@ -601,7 +607,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2) gemv1_kernel(const __grid_cons
     const uint4* xp = reinterpret_cast<const uint4*>(xs + (size_t)uc * kXw);
 #pragma unroll
     for (int i = 0; i < kXw / 4; ++i) {
-      const uint4 v = xp[i ^ (half_first * (kXw / 8))];
+      const uint4 v = xp[(i ^ (half_first * (kXw / 8))) ^ (uc & (kXw / 4 - 1))];
       xr[4 * i] = v.x;
       xr[4 * i + 1] = v.y;
       xr[4 * i + 2] = v.z;
