@@ -118,3 +118,29 @@ def test_quantize_validation_returns_before_launch(lib):
     assert lib.qlin_quantize_rtn(Q.Desc(64, 100, 4).ref(), p, p, p, p, p, None) == -3
     assert lib.qlin_quantize_rtn(Q.Desc(64, 128, 5).ref(), p, p, p, p, p, None) == -2
     assert lib.qlin_quantize_rtn(Q.Desc(65, 128, 0, [6, 6]).ref(), p, p, p, p, p, None) == -3
+
+
+def test_binding_rejects_host_tensors(lib):
+    """Every entry point of the binding takes CUDA tensors only and raises for
+    host tensors before calling the library: there is no CPU path."""
+    import torch
+    d = Q.Desc(64, 128, 4)
+    h16 = torch.zeros(64, 128, dtype=torch.float16)
+    s = torch.zeros(64, 1, dtype=torch.float16)
+    sb = torch.zeros(4, dtype=torch.int32)
+    x = torch.zeros(1, 128, dtype=torch.float16)
+    packed = torch.zeros(Q.qlin_packed_bytes(d), dtype=torch.uint8)
+    calls = [
+        lambda: Q.qlin_pack(d, torch.zeros(64, 128, dtype=torch.uint8), packed),
+        lambda: Q.qlin_unpack(d, packed, torch.zeros(64, 128, dtype=torch.uint8)),
+        lambda: Q.qlin_dequant(d, packed, s, s, h16),
+        lambda: Q.qlin_rht(x, sb, torch.zeros_like(x)),
+        lambda: Q.qlin_quantize_rtn(d, h16, sb, torch.zeros(64, 128, dtype=torch.uint8), s.clone(), s.clone()),
+        lambda: Q.qlin_gemv(d, packed, s, s, sb, x, torch.zeros(1, 64, dtype=torch.float16),
+                            torch.zeros(256, dtype=torch.uint8)),
+        lambda: Q.qlin_gemm(d, packed, s, s, sb, x, torch.zeros(1, 64, dtype=torch.float16),
+                            torch.zeros(1 << 16, dtype=torch.uint8)),
+    ]
+    for call in calls:
+        with pytest.raises(TypeError, match="CUDA tensor"):
+            call()
