@@ -470,9 +470,9 @@ def case_host_packed(case_host, bits, block_bits):
     return _PACKED_CACHE[key]
 
 
-def cpu_quantize_rate(case: Case, budget_s: float = 12.0):
+def cpu_quantize_rate(case: Case, budget_s: float = 12.0, threads: int | None = 1):
     """Oracle throughput of the offline tool (GB/s of its algorithmic bytes) on
-    row samples of the weight, BLAS limited to one thread."""
+    row samples of the weight, BLAS limited to `threads` (None: all cores)."""
     from threadpoolctl import threadpool_limits
     from oracle import qlin_oracle as O
     w, sb = case.host_sample
@@ -480,7 +480,7 @@ def cpu_quantize_rate(case: Case, budget_s: float = 12.0):
     per_row = case.bytes / N
     rng = np.random.default_rng(0)
     done_rows, t = 0, 0.0
-    with threadpool_limits(limits=1):
+    with threadpool_limits(limits=threads):
         while t < budget_s and done_rows < N:
             rows = np.sort(rng.choice(N, size=min(256, N), replace=False))
             t1 = time.perf_counter()
@@ -490,9 +490,11 @@ def cpu_quantize_rate(case: Case, budget_s: float = 12.0):
     return done_rows * per_row / t / 1e9, done_rows, t
 
 
-def cpu_oracle_rate(case: Case, budget_s: float = 12.0, rows_per_step: int | None = None):
+def cpu_oracle_rate(case: Case, budget_s: float = 12.0, rows_per_step: int | None = None,
+                    threads: int | None = 1):
     """Oracle throughput (GB/s of the layer's algorithmic bytes) on a bounded
-    sample of the workload's weight rows, BLAS limited to one thread."""
+    sample of the workload's weight rows, BLAS limited to `threads` (None: all
+    cores)."""
     from threadpoolctl import threadpool_limits
     from oracle import qlin_oracle as O
     codes = case.host_sample[0]
@@ -501,7 +503,7 @@ def cpu_oracle_rate(case: Case, budget_s: float = 12.0, rows_per_step: int | Non
     case_host_packed(case.host_sample, case.bits, bb)
     per_row = O.algorithmic_bytes(N, K, case.bits or None, bb) / N
     rng = np.random.default_rng(0)
-    with threadpool_limits(limits=1):
+    with threadpool_limits(limits=threads):
         t0 = time.perf_counter()
         rows = np.sort(rng.choice(N, size=min(64, N), replace=False))
         oracle_step(case.host_sample, rows, case.bits, bb)
@@ -563,7 +565,7 @@ def run_ours(args):
     roof["algorithmic_bytes_per_launch"] = case.bytes
     e2e = None if args.no_extras else time_e2e(case, args.steps, args.warmup, stream)
     cublas_us = time_cublas(case, stream) if rank == 0 and not args.no_extras else None
-    cpu = None
+    cpu = cpu_all = None
     if rank == 0 and world == 1 and case.host_sample is not None and not args.no_cpu_baseline \
             and not args.no_extras:
         if case.kind == "quantize":
@@ -574,6 +576,12 @@ def run_ours(args):
             what = "unpack + fp64 dequant + explicit-H rotation + fp64 matmul"
         cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": f"{rows} of {case.N} weight rows ({what}), {t:.1f} s, BLAS limited to 1 thread"}
+        # the same oracle with BLAS on every host core (the unpack/dequant steps stay single-threaded numpy)
+        ncores = os.cpu_count() or 1
+        rate = cpu_quantize_rate if case.kind == "quantize" else cpu_oracle_rate
+        gbs_all, rows_all, t_all = rate(case, budget_s=args.cpu_budget / 2, threads=None)
+        cpu_all = {"value": gbs_all, "unit": "GB/s", "cores": ncores, "kind": "oracle",
+                   "sample": f"{rows_all} of {case.N} weight rows ({what}), {t_all:.1f} s, BLAS on {ncores} threads"}
     if rank == 0:
         us = ms_step * 1e3
         cfg = {"workload": case.desc_text, "M": case.M, "K": case.K, "N": case.N,
@@ -590,6 +598,8 @@ def run_ours(args):
                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                "dtype": "f64" if case.kind == "quantize" else "f16", "data": "synthetic", "config": cfg, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                "gpu_launches": case.launches_per_step() * args.steps, "clocks": clocks}
+        if cpu_all is not None:
+            out["cpu_baseline_all_cores"] = cpu_all
         if cublas_us is not None:
             out["cublas_bf16"] = {"us_per_call": cublas_us, "speedup": cublas_us / us}
         if no_overlap is not None:
