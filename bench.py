@@ -481,7 +481,7 @@ def cpu_quantize_rate(case: Case, budget_s: float = 12.0, threads: int | None = 
     rng = np.random.default_rng(0)
     done_rows, t = 0, 0.0
     with threadpool_limits(limits=threads):
-        while t < budget_s and done_rows < N:
+        while t < budget_s and done_rows < 32 * N:
             rows = np.sort(rng.choice(N, size=min(256, N), replace=False))
             t1 = time.perf_counter()
             O.quantize_rtn(w[rows], sb, case.bits)
@@ -510,15 +510,14 @@ def cpu_oracle_rate(case: Case, budget_s: float = 12.0, rows_per_step: int | Non
         t_row = (time.perf_counter() - t0) / len(rows)
         if rows_per_step is None:
             rows_per_step = int(max(16, min(N, budget_s / max(t_row, 1e-9))))
+        # samples of rows_per_step rows until the time budget is spent (at most 32 passes' worth)
         done_rows, t = 0, 0.0
-        while t < budget_s and done_rows < 4 * N:
+        while t < budget_s and done_rows < 32 * N:
             rows = np.sort(rng.choice(N, size=min(rows_per_step, N), replace=False))
             t1 = time.perf_counter()
             oracle_step(case.host_sample, rows, case.bits, bb)
             t += time.perf_counter() - t1
             done_rows += len(rows)
-            if rows_per_step is not None and t > 0 and done_rows >= rows_per_step:
-                break
     gbs = done_rows * per_row / t / 1e9
     return gbs, done_rows, t
 
