@@ -204,7 +204,8 @@ size_t qlin_gemv_workspace_bytes(const qlin_desc* desc, int32_t M);
  * scale per 64 (int8: 32) consecutive values: exact for values within a
  * factor 16 of the largest magnitude of their run, others rounded at 2^-14 of
  * it.  These readings are judged by the output tolerance, like the factored
- * scale.
+ * scale.  For 2 <= M <= 16 (and mixed widths) x is rotated into the workspace
+ * and the codes, exact as fp16, are multiplied with it on the tensor cores.
  *   x : device fp16 [M][K] (not rotated);  y : device fp16 [M][N];
  *   workspace : device buffer of workspace_bytes >= qlin_gemv_workspace_bytes(M, K)
  *               bytes (may be NULL when that is 0); overwritten.
@@ -216,14 +217,16 @@ qlin_status qlin_gemv(const qlin_desc* desc, const void* packed, const uint16_t*
                       uint16_t* y, int32_t M, void* workspace, size_t workspace_bytes,
                       qlin_stream_t stream);
 
-/* Workspace bytes qlin_gemm needs for this weight and M (the rotated
- * activations, M*K fp16, rounded up to 256 bytes). */
+/* Workspace bytes qlin_gemm needs for this weight and M: the rotated
+ * activations (M*K fp16, rounded up to 256 bytes), the completion flags of the
+ * work split between CTAs, and one fp32 partial tile per CTA. */
 size_t qlin_gemm_workspace_bytes(const qlin_desc* desc, int32_t M);
 
 /* Prefill-regime quantised linear layer, any M >= 1 (built for M >= 64):
  * same result definition as qlin_gemv, with the weight dequantised exactly as
- * qlin_dequant does into shared memory and multiplied on the tensor cores
- * (fp16 operands, fp32 accumulation).
+ * qlin_dequant does into tensor memory and multiplied on the tensor cores
+ * (fp16 operands, fp32 accumulation).  Tiles split between CTAs are summed in
+ * a fixed order, so the result is deterministic.
  *   workspace : device buffer of workspace_bytes >= qlin_gemm_workspace_bytes(M, K)
  *               bytes; overwritten. */
 qlin_status qlin_gemm(const qlin_desc* desc, const void* packed, const uint16_t* scales,
