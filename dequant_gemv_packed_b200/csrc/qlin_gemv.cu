@@ -67,7 +67,8 @@ constexpr int kPartialBudget = 24 * 1024;
 constexpr int kMaxStages = 16;
 constexpr int kSms = 148;
 
-template <int N> struct int_ { static constexpr int value = N; };
+template <int N> struct int_ {};
+template <int N> struct rows_ { static constexpr int value = N; };  // rows a lane takes in one pass
 
 // A unit is the run of codes one lane multiplies with its x registers.
 template <int B> struct UnitT;
@@ -662,12 +663,12 @@ __global__ void __launch_bounds__(kMaxThreads, 2) gemv1_kernel(const __grid_cons
     for (int rb = 0; rb < cr;) {
       if constexpr (B != 8) {
         if (cr - rb <= (R - 1) * RS) {
-          pass(rb, int_<1>{});
+          pass(rb, rows_<1>{});
           rb += RS;
           continue;
         }
       }
-      pass(rb, int_<R>{});
+      pass(rb, rows_<R>{});
       rb += R * RS;
     }
     if (ring) {
