@@ -184,6 +184,15 @@ static qlin_status check_linear(const qlin_desc* d, const void* packed, const ui
   return QLIN_OK;
 }
 
+qlin_status qlin_gemv_plan(const qlin_desc* d, int32_t M, qlin_gemv_plan_info* info) {
+  qlin_status r = check_desc(d);
+  if (r != QLIN_OK) return r;
+  if (!info) return QLIN_ERR_INVALID_ARG;
+  if (M < 1 || M > 16) return QLIN_ERR_SHAPE;
+  gemv_plan_info(d->bits, d->N, d->K, M, info);
+  return QLIN_OK;
+}
+
 size_t qlin_gemv_workspace_bytes(const qlin_desc* d, int32_t M) {
   if (check_desc(d) != QLIN_OK || M < 1 || M > 16) return 0;
   return gemv_workspace_bytes(d->bits, d->N, d->K, M);

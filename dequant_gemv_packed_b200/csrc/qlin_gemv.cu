@@ -1202,6 +1202,29 @@ qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half*
   return record_cuda(cudaGetLastError());
 }
 
+void gemv_plan_info(int bits, int N, int K, int M, qlin_gemv_plan_info* info) {
+  *info = qlin_gemv_plan_info{};
+  Plan p;
+  if (M == 1 && bits != 0 && make_plan(bits, N, K, p)) {
+    info->kernel = 1;
+    info->grid = p.grid;
+    info->threads = (p.NW + 1) * 32;
+    info->smem_bytes = p.smem_bytes;
+    info->consumer_warps = p.NW;
+    info->units_per_warp = p.UW;
+    info->rows_per_cta = p.rows_per_cta;
+    info->rows_per_chunk = p.rows_per_chunk;
+    info->stages = p.stages;
+    info->chunks_in_flight = p.inflight;
+    return;
+  }
+  const MmaWorkspace ws(N, K, M);
+  info->kernel = 2;
+  info->grid = ws.grid;
+  info->threads = 32 * ws.warps_per_block;
+  info->workspace_bytes = ws.total;
+}
+
 unsigned take_gemv_error() {
   unsigned v = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&v, g_gemv_error, sizeof(v)) != cudaSuccess) return ~0u;

@@ -48,6 +48,7 @@ qlin_status launch_dequant(const PackedView& v, const __half* scales, const __ha
 qlin_status launch_rht(const __half* x, __half* xr, const uint32_t* sign_bits, int M, int K,
                        cudaStream_t s, uint32_t* clear = nullptr, int nclear = 0, float* xsum = nullptr);
 size_t gemv_workspace_bytes(int bits, int N, int K, int M);
+void gemv_plan_info(int bits, int N, int K, int M, qlin_gemv_plan_info* info);
 unsigned take_gemv_error();
 unsigned take_gemm_error();
 qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half* zeros,

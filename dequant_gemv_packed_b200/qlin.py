@@ -23,7 +23,7 @@ EXPORTED = (
     "qlin_status_string", "qlin_last_cuda_error", "qlin_packed_bytes", "qlin_code_bytes", "qlin_pack",
     "qlin_unpack", "qlin_dequant", "qlin_rht", "qlin_gemv_workspace_bytes", "qlin_gemv",
     "qlin_gemm_workspace_bytes", "qlin_gemm", "qlin_device_error", "qlin_gemm_noalloc", "qlin_set_overlap",
-    "qlin_quantize_rtn",
+    "qlin_quantize_rtn", "qlin_gemv_plan",
 )
 
 
@@ -85,6 +85,7 @@ def lib() -> ctypes.CDLL:
     L.qlin_dequant.argtypes, L.qlin_dequant.restype = [vp, vp, vp, vp, vp, vp], ctypes.c_int
     L.qlin_rht.argtypes, L.qlin_rht.restype = [vp, vp, vp, i32, i32, vp], ctypes.c_int
     L.qlin_quantize_rtn.argtypes, L.qlin_quantize_rtn.restype = [vp, vp, vp, vp, vp, vp, vp], ctypes.c_int
+    L.qlin_gemv_plan.argtypes, L.qlin_gemv_plan.restype = [vp, i32, vp], ctypes.c_int
     L.qlin_gemv_workspace_bytes.argtypes, L.qlin_gemv_workspace_bytes.restype = [vp, i32], sz
     L.qlin_gemm_workspace_bytes.argtypes, L.qlin_gemm_workspace_bytes.restype = [vp, i32], sz
     L.qlin_device_error.argtypes, L.qlin_device_error.restype = [ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int
@@ -188,6 +189,19 @@ def qlin_dequant(desc: Desc, packed: torch.Tensor, scales: torch.Tensor, zeros: 
                               _dev(zeros, torch.float16, "zeros"), _dev(w, torch.float16, "w"), _stream(stream)),
            "qlin_dequant")
     return w
+
+
+class _GemvPlan(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_int32) for name in (
+        "kernel", "grid", "threads", "smem_bytes", "consumer_warps", "units_per_warp", "rows_per_cta",
+        "rows_per_chunk", "stages", "chunks_in_flight")] + [("workspace_bytes", ctypes.c_uint64)]
+
+
+def qlin_gemv_plan(desc: Desc, M: int) -> dict:
+    """The launch plan qlin_gemv uses for this weight and M (host only)."""
+    info = _GemvPlan()
+    _check(lib().qlin_gemv_plan(desc.ref(), M, ctypes.byref(info)), "qlin_gemv_plan")
+    return {name: getattr(info, name) for name, _ in _GemvPlan._fields_}
 
 
 def qlin_quantize_rtn(desc: Desc, w: torch.Tensor, sign_bits: torch.Tensor, codes: Optional[torch.Tensor] = None,

@@ -187,6 +187,29 @@ qlin_status qlin_quantize_rtn(const qlin_desc* desc, const uint16_t* w, const ui
 qlin_status qlin_rht(const uint16_t* x, uint16_t* xr, const uint32_t* sign_bits, int32_t M,
                      int32_t K, qlin_stream_t stream);
 
+/* Launch plan of qlin_gemv for this weight and M, computed on the host
+ * without launching anything: which kernel runs and how it is laid out (for
+ * capacity planning, e.g. whether consecutive calls' CTAs fit on an SM
+ * together).  Fields a kernel does not have are 0. */
+typedef struct {
+  int32_t kernel;           /* 1: fused M = 1 kernel (uniform widths);
+                               2: rotation kernel + tensor-core kernel          */
+  int32_t grid;             /* CTAs of the main kernel                         */
+  int32_t threads;          /* threads per CTA                                 */
+  int32_t smem_bytes;       /* dynamic shared memory per CTA                   */
+  int32_t consumer_warps;   /* kernel 1: warps that multiply (plus 1 producer) */
+  int32_t units_per_warp;   /* kernel 1: runs of 64 codes (8-bit: 32) per warp */
+  int32_t rows_per_cta;     /* kernel 1: the most rows one CTA owns            */
+  int32_t rows_per_chunk;   /* kernel 1: rows one bulk copy brings in          */
+  int32_t stages;           /* kernel 1: shared-memory stages                  */
+  int32_t chunks_in_flight; /* kernel 1: copies of one CTA in flight at once   */
+  uint64_t workspace_bytes; /* = qlin_gemv_workspace_bytes(desc, M)            */
+} qlin_gemv_plan_info;
+
+/* Fills *info; QLIN_ERR_INVALID_ARG / _UNSUPPORTED / _SHAPE as qlin_gemv
+ * (M outside 1..16). */
+qlin_status qlin_gemv_plan(const qlin_desc* desc, int32_t M, qlin_gemv_plan_info* info);
+
 /* Workspace bytes qlin_gemv needs for this weight and M; 0 means none (the
  * workspace may then be NULL).  Returns 0 for an invalid descriptor or M. */
 size_t qlin_gemv_workspace_bytes(const qlin_desc* desc, int32_t M);

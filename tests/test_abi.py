@@ -144,3 +144,46 @@ def test_binding_rejects_host_tensors(lib):
     for call in calls:
         with pytest.raises(TypeError, match="CUDA tensor"):
             call()
+
+
+def test_gemv_plan_invariants(lib):
+    """Launch plans of qlin_gemv over a sweep of widths, K and N (host only):
+    the invariants the kernels' index bounds rely on."""
+    Ns = (1, 2, 63, 64, 147, 148, 149, 1000, 2560, 4096, 4737, 9728, 19456, 151936, 262144)
+    smem_floor, smem_limit = 80 * 1024, 113 * 1024
+    for bits in (3, 4, 6, 8):
+        unit = 32 if bits == 8 else 64
+        rows_per_pass = 4 if bits == 4 else 2
+        for K in list(range(128, 4097, 128)) + [5120, 9728, 12288, 16384, 20480, 24576, 32768]:
+            for N in Ns:
+                d = Q.Desc(N, K, bits)
+                p = Q.qlin_gemv_plan(d, 1)
+                assert p["workspace_bytes"] == Q.qlin_gemv_workspace_bytes(d, 1)
+                if p["kernel"] == 2:  # very long K: the tensor-core kernel with a workspace
+                    assert K // unit > 320 and p["workspace_bytes"] > 0
+                    continue
+                U, NW, UW = K // unit, p["consumer_warps"], p["units_per_warp"]
+                assert 1 <= NW <= 10 and UW in (1, 2, 4, 8, 16, 32) and (NW - 1) * UW < U <= NW * UW
+                assert p["threads"] == 32 * (NW + 1)
+                assert smem_floor <= p["smem_bytes"] <= smem_limit, (bits, K, N, p)
+                assert p["grid"] == min(148, N) and p["rows_per_cta"] == -(-N // p["grid"])
+                assert p["rows_per_chunk"] % (rows_per_pass * 32 // UW) == 0
+                nchunks = -(-p["rows_per_cta"] // p["rows_per_chunk"])
+                assert 1 <= p["stages"] <= min(16, nchunks) and 1 <= p["chunks_in_flight"] <= p["stages"]
+                row_bytes = K * bits // 8
+                resident = p["rows_per_cta"] if p["stages"] == nchunks else p["stages"] * p["rows_per_chunk"]
+                assert resident * row_bytes < p["smem_bytes"], (bits, K, N, p)
+    for M in (2, 16):
+        p = Q.qlin_gemv_plan(Q.Desc(2560, 9728, 3), M)
+        assert p["kernel"] == 2 and p["workspace_bytes"] == Q.qlin_gemv_workspace_bytes(Q.Desc(2560, 9728, 3), M)
+    p = Q.qlin_gemv_plan(Q.Desc(320, 1280, 0, [6, 8, 4, 3, 8]), 1)
+    assert p["kernel"] == 2  # mixed widths
+
+
+def test_gemv_plan_validation(lib):
+    info = ctypes.create_string_buffer(64)
+    assert lib.qlin_gemv_plan(Q.Desc(64, 128, 4).ref(), 17, info) == -3
+    assert lib.qlin_gemv_plan(Q.Desc(64, 128, 4).ref(), 0, info) == -3
+    assert lib.qlin_gemv_plan(Q.Desc(64, 128, 4).ref(), 1, None) == -1
+    assert lib.qlin_gemv_plan(Q.Desc(64, 100, 4).ref(), 1, info) == -3
+    assert lib.qlin_gemv_plan(None, 1, info) == -1
