@@ -268,14 +268,6 @@ def linear64(x: np.ndarray, codes: np.ndarray, scales: np.ndarray, zeros: np.nda
     return xr @ w.T
 
 
-def linear_strict(x: np.ndarray, codes: np.ndarray, scales: np.ndarray, zeros: np.ndarray,
-                  sign_bits: np.ndarray) -> np.ndarray:
-    """Diagnostic: the same sum over fp16-rounded x~ and fp16 weights (fp64 sum)."""
-    xr = rht16(x, sign_bits).astype(np.float64)
-    w = dequant16(codes, scales, zeros).astype(np.float64)
-    return xr @ w.T
-
-
 def algorithmic_bytes(N: int, K: int, bits: int | None = None, block_bits=None) -> int:
     """Bytes a kernel must read from memory for one pass over the weight:
     packed codes plus the fp16 scale and zero of every group (plus one selector

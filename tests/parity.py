@@ -44,11 +44,12 @@ def assert_close(y, y_ref, what=""):
     return rel_max, rel_fro
 
 
-def assert_close_abs(y, w, a, rows=None, what=""):
-    """Degenerate outputs (fewer than 16 values): a single dot product can cancel
-    to far below its terms, so the spec's relative-to-max|y| bound says nothing
-    about the kernel there.  Use the standard dot-product bound instead:
-    |y - y_ref| <= 2e-3 * sum_k |x~_k w_k| (fp64 oracle terms)."""
+def assert_dot_bound(y, w, a, rows=None, what=""):
+    """Extra per-element check beside the output tolerance: every output is a
+    dot product of K terms, and its error is held to 2e-3 of the sum of the
+    terms' magnitudes, |y - y_ref| <= 2e-3 * sum_k |x~_k w_k| (fp64 oracle
+    terms).  Unlike the max-relative bound it does not depend on the other
+    outputs, so it also bounds outputs that cancel to far below their terms."""
     rows = np.arange(w.N) if rows is None else np.asarray(rows)
     t = torch.as_tensor(rows, device=w.codes.device)
     xr = O.rht64(a.x.cpu().numpy(), np_u32(a.sign_bits))
