@@ -31,6 +31,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "qlin_internal.cuh"
@@ -601,15 +602,19 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+EncodeTiledFn lookup_encode_fn() {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<EncodeTiledFn>(p);
+  return nullptr;
+}
+
+// The driver's tensor-map encoder, looked up once (a function-local static is
+// initialised exactly once even when several host threads call at once).
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+  static const EncodeTiledFn fn = lookup_encode_fn();
   return fn;
 }
 
@@ -675,14 +680,17 @@ qlin_status launch_gemm_rotated(const PackedView& v, const __half* scales, const
     ymap = map;  // unused
   }
 
-  static unsigned long long configured = 0;
+  // One bit per device: the attribute is set once per device.  Host threads
+  // making their first call together may both set it (harmless); the bits are
+  // atomic, so there is no data race.
+  static std::atomic<unsigned long long> configured{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return record_cuda(e);
-  if (dev >= 64 || !((configured >> dev) & 1ull)) {
+  if (dev >= 64 || !((configured.load(std::memory_order_acquire) >> dev) & 1ull)) {
     e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return record_cuda(e);
-    if (dev < 64) configured |= 1ull << dev;
+    if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_release);
   }
   const long long tiles = (long long)a.m_tiles * a.n_tiles;
   const long long work = a.stream_k ? tiles * (v.K / kGroup) : tiles;

@@ -43,6 +43,7 @@
 //     under this call's arithmetic.
 // Other cases (M > 1, mixed widths, very long K): gemv_mma_kernel below.
 #include <algorithm>
+#include <atomic>
 
 #include "qlin_internal.cuh"
 #include "qlin_sm100.cuh"
@@ -800,11 +801,13 @@ bool make_plan(int b, int N, int K, Plan& p) {
 
 template <int B, int UW>
 qlin_status launch_gemv1_uw(const Args& a, cudaStream_t s) {
-  static unsigned long long configured = 0;  // one bit per device (the attribute is per device)
+  // One bit per device (the attributes are per device), atomic: host threads
+  // making their first call together may both set the attributes (harmless).
+  static std::atomic<unsigned long long> configured{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return record_cuda(e);
-  if (dev >= 64 || !((configured >> dev) & 1ull)) {
+  if (dev >= 64 || !((configured.load(std::memory_order_acquire) >> dev) & 1ull)) {
     e = cudaFuncSetAttribute(gemv1_kernel<B, UW>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     if (e != cudaSuccess) return record_cuda(e);
     // Every instance asks for the largest shared-memory carveout, so that
@@ -813,7 +816,7 @@ qlin_status launch_gemv1_uw(const Args& a, cudaStream_t s) {
     e = cudaFuncSetAttribute(gemv1_kernel<B, UW>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return record_cuda(e);
-    if (dev < 64) configured |= 1ull << dev;
+    if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.p.grid);

@@ -121,10 +121,17 @@ int qlin_last_cuda_error(void);
 int qlin_set_overlap(int enable);
 
 /* Bytes of the packed buffer for `desc` (codes, plus the block table for mixed
- * widths), a multiple of 16.  Returns 0 for an invalid descriptor. */
+ * widths), a multiple of 16.  Returns 0 for an invalid descriptor.  Counts the
+ * stored format: K*b/8 bytes per row of b-bit codes ("24B0978-Week01-Track2_20-
+ * Submission01", paragraph "Group-wise affine integer quantisation"; mixed
+ * widths per 64-row block: "25M2111-Week02-Track2-40-Submission01", section
+ * "Method, selection, and reproduction"). */
 size_t qlin_packed_bytes(const qlin_desc* desc);
 
-/* Bytes of the code stream alone (the layout above without the block table). */
+/* Bytes of the code stream alone (the layout above without the block table):
+ * the packed codes that one pass over the weight reads, the bulk of the weight
+ * traffic that the pages' decode speed-up rests on ("24B0978-Week01-Track2_20-
+ * Submission01", section "How these techniques accelerate inference on CUDA"). */
 size_t qlin_code_bytes(const qlin_desc* desc);
 
 /* Pack integer codes into the layout above.
@@ -137,7 +144,10 @@ qlin_status qlin_pack(const qlin_desc* desc, const uint8_t* codes, void* packed,
                       qlin_stream_t stream);
 
 /* Inverse of qlin_pack: codes (device uint8 [N][K]) from a packed buffer.
- * Uses the same device decode routines as qlin_gemv and qlin_gemm. */
+ * Uses the same device decode routines as qlin_gemv and qlin_gemm.
+ * Definition: the layout above ("24B0978-Week01-Track2_20-Submission01",
+ * paragraph "Group-wise affine integer quantisation": integer codes per group
+ * of 128 along K). */
 qlin_status qlin_unpack(const qlin_desc* desc, const void* packed, uint8_t* codes,
                         qlin_stream_t stream);
 
@@ -242,14 +252,22 @@ qlin_status qlin_gemv(const qlin_desc* desc, const void* packed, const uint16_t*
 
 /* Workspace bytes qlin_gemm needs for this weight and M: the rotated
  * activations (M*K fp16, rounded up to 256 bytes), the completion flags of the
- * work split between CTAs, and one fp32 partial tile per CTA. */
+ * work split between CTAs, and one fp32 partial tile per CTA.  The rotated
+ * activations are the runtime half of the random Hadamard transform
+ * ("24B0978-Week01-Track2_20-Submission01", paragraph "Random Hadamard
+ * transform"), computed once per call and read by every CTA. */
 size_t qlin_gemm_workspace_bytes(const qlin_desc* desc, int32_t M);
 
 /* Prefill-regime quantised linear layer, any M >= 1 (built for M >= 64):
- * same result definition as qlin_gemv, with the weight dequantised exactly as
- * qlin_dequant does into tensor memory and multiplied on the tensor cores
- * (fp16 operands, fp32 accumulation).  Tiles split between CTAs are summed in
- * a fixed order, so the result is deterministic.
+ *   y[m][n] = fp16_rn( sum_k rht(x)[m][k] * w[n][k] ), fp32 accumulation,
+ * with rht(x) rounded once to fp16 and w the fp16 weight exactly as
+ * qlin_dequant writes it, dequantised into tensor memory inside the main loop
+ * and multiplied on the tensor cores (fp16 operands, fp32 accumulation); the
+ * fp16 weight never reaches global memory.  Tiles split between CTAs are
+ * summed in a fixed order, so the result is deterministic.
+ * Definition: "24B0978-Week01-Track2_20-Submission01", section "How these
+ * techniques accelerate inference on CUDA" (dequantisation fused into the
+ * matmul; group-wise affine codes; activation rotation at runtime).
  *   workspace : device buffer of workspace_bytes >= qlin_gemm_workspace_bytes(M, K)
  *               bytes; overwritten. */
 qlin_status qlin_gemm(const qlin_desc* desc, const void* packed, const uint16_t* scales,
@@ -258,7 +276,12 @@ qlin_status qlin_gemm(const qlin_desc* desc, const void* packed, const uint16_t*
                       qlin_stream_t stream);
 
 /* qlin_gemm for callers that cannot allocate device memory: the pages have no
- * counterpart; this is a library convenience.  qlin_gemm needs a workspace for
+ * counterpart; this is a library convenience.  It has no room for the partial
+ * sums of tiles split between CTAs, so it runs the one-CTA-per-tile schedule
+ * (each output tile summed over all of K by one CTA): the same result
+ * definition as qlin_gemm within the output tolerance, but a different
+ * summation order (not bit-identical to qlin_gemm) and slower when there are
+ * fewer tiles than SMs.  qlin_gemm needs a workspace for
  * the rotated activations, but some callers cannot allocate one where they run
  * the layer (for example a plugin inside another runtime that owns all device
  * allocations, or a serving loop that forbids allocation once running, since

@@ -6,8 +6,11 @@ allocation once running) use qlin_gemm_noalloc, which keeps the rotated
 activations in an array inside the library instead of a caller workspace.
 This test calls it through the C ABI twice in a row, with different shapes so
 that stale contents of the shared array would show, and compares each result
-with qlin_gemm's on the same inputs, within the parity tolerances.  It lives in
-a file of its own that pytest collects last.
+with qlin_gemm's on the same inputs and with the CPU oracle, within the parity
+tolerances.  qlin_gemm_noalloc has no workspace for split tiles, so it runs the
+one-CTA-per-tile schedule (each output tile summed by one CTA over all of K);
+the oracle comparison is what checks that schedule.  It lives in a file of its
+own that pytest collects last.
 """
 import ctypes
 
@@ -60,6 +63,10 @@ def test_noalloc_matches_gemm_on_two_calls():
         assert np.isfinite(got).all()
         rel_max, rel_fro = O.parity_errors(got, ref)
         assert rel_max <= MAX_REL and rel_fro <= FRO_REL, (M, N, K, rel_max, rel_fro)
+        oracle = O.linear64(a.x.cpu().numpy(), w.codes.cpu().numpy(), w.scales.cpu().numpy(),
+                            w.zeros.cpu().numpy(), a.sign_bits.cpu().numpy().view(np.uint32))
+        rel_max, rel_fro = O.parity_errors(got, oracle)
+        assert rel_max <= MAX_REL and rel_fro <= FRO_REL, ("oracle", M, N, K, rel_max, rel_fro)
     assert Q.qlin_device_error() == 0
 
 
