@@ -307,6 +307,9 @@ class Case:
         self.call(self.d, packed, s, z, self.sign_bits, self.x, self.y[i % self.copies], self.ws)
 
 
+SPIN_CYCLES = 200_000  # ~0.1 ms at 1.9 GHz, longer than the host needs to queue the timed replays
+
+
 def time_steps(case: Case, K: int, W: int, dist, stream, graph_len: int = 1024):
     """Warm up W steps, then time exactly K steps replayed from CUDA graphs."""
     torch.cuda.synchronize()
@@ -330,9 +333,10 @@ def time_steps(case: Case, K: int, W: int, dist, stream, graph_len: int = 1024):
                 for i in range(rem):
                     case.step(R + i)
             graphs.append((g2, rem))
-        # one untimed replay of each graph (uploads the graph)
-        for g_, _ in graphs:
-            g_.replay()
+        # untimed replays of each graph (uploads the graph; warms clocks and caches)
+        for _ in range(3):
+            for g_, _ in graphs:
+                g_.replay()
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(dist)
@@ -340,6 +344,11 @@ def time_steps(case: Case, K: int, W: int, dist, stream, graph_len: int = 1024):
     sampler = ClockSampler(torch.cuda.current_device())
     with sampler:
         with torch.cuda.stream(stream):
+            # A short device-side spin ahead of the start event: the host queues
+            # the graph replays while it runs, so the timed region holds the K
+            # steps back to back and no host enqueue gap (which a 20-step run
+            # would otherwise spread over only 20 calls).
+            torch.cuda._sleep(SPIN_CYCLES)
             torch.cuda.nvtx.range_push("qlin_timed")
             start.record(stream)
             for _ in range(K // R):

@@ -46,6 +46,7 @@
 #include <atomic>
 
 #include "qlin_internal.cuh"
+#include "qlin_rot16.cuh"
 #include "qlin_sm100.cuh"
 
 namespace qlin {
@@ -363,13 +364,6 @@ __device__ __forceinline__ int group_add(int v, int grp) {
   return r;
 }
 
-// (H[r][c], H[r][c+1]) of the Sylvester matrix of order 16 as two fp16 (+-1).
-__device__ __forceinline__ uint32_t h16_pair(int r, int c) {
-  const uint32_t lo = (__popc(r & c) & 1) ? 0xBC00u : 0x3C00u;
-  const uint32_t hi = (__popc(r & (c + 1)) & 1) ? 0xBC00u : 0x3C00u;
-  return lo | (hi << 16);
-}
-
 // Position in dp2a order of code c of a 64-code int4 unit (pairs (0,2) (4,6)
 // (1,3) (5,7) of each word of 8 codes; see dot_unit_int).
 __device__ __forceinline__ int int4_slot(int c) {
@@ -383,45 +377,20 @@ __device__ __forceinline__ int int4_slot(int c) {
 // banks.  x_half maps a 16-bit position of the unit to its place.
 __device__ __forceinline__ int x_half(int p, int u, int P) { return (((p >> 3) ^ (u & (P - 1))) << 3) | (p & 7); }
 
-// Sign flip, block-128 FWHT, x 1/sqrt(128) and fp16 rounding of one block,
-// then the unit preparation described at the top of the file.
-// The order-128 Sylvester matrix is H16 (x) H8 (element e = i + 16 j: bits
-// 0-3 and 4-6 of e), so with X[i][j] = d_e x_e the rotation is H16 X H8: one
-// m16n8k16 tensor-core product (A = H16, B = X) and three butterfly stages
-// along j.  Lane (g, t) = (lane / 4, lane % 4) supplies X[2t, 2t+1][g] and
-// X[2t+8, 2t+9][g] (x at 16g + 2t and 16g + 2t + 8: b0 and b1, signs in sw)
-// and ends with elements g + 32t + {0, 16, 8, 24}.
+// Sign flip, block-128 FWHT, x 1/sqrt(128) and fp16 rounding of one block
+// (rotate_block16x8: one tensor-core product with H16, butterflies along H8),
+// then the unit preparation described at the top of the file.  Lane (g, t)
+// ends with elements g + 32t + {0, 16, 8, 24}.
 template <int B>
 __device__ __forceinline__ void rotate_prepare(uint32_t b0, uint32_t b1, uint32_t sw, int blk, bool store,
                                                const uint32_t (&h)[4], uint32_t* xs, float2* ust, int lane) {
   using UT = UnitT<B>;
   constexpr int kXw = UT::kCodes / 2;
   const int g = lane >> 2, t = lane & 3;
-  b0 ^= ((sw & 1u) << 15) | ((sw & 2u) << 30);
-  b1 ^= (((sw >> 8) & 1u) << 15) | (((sw >> 8) & 2u) << 30);
-  float c0, c1, c2, c3;
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
-      : "=f"(c0), "=f"(c1), "=f"(c2), "=f"(c3)
-      : "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3]), "r"(b0), "r"(b1), "f"(0.f));
-  // columns 2t, 2t+1 (stride 1 in j), then partners t^1 and t^2 (strides 2, 4)
-  float v[4] = {c0 + c1, c0 - c1, c2 + c3, c2 - c3};
-#pragma unroll
-  for (int o = 1; o <= 2; o <<= 1) {
-    const bool up = (t & o) != 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float q = __shfl_xor_sync(0xffffffffu, v[i], o);
-      v[i] = up ? q - v[i] : v[i] + q;
-    }
-  }
-  constexpr int kOff[4] = {0, 16, 8, 24};  // element of v[i]: g + 32 t + kOff[i]
   __half hv[4];
   float f[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    hv[i] = __float2half_rn(v[i] * kInvSqrt128);
-    f[i] = __half2float(hv[i]);
-  }
+  rotate_block16x8(b0, b1, sw, h, lane, hv, f);
+  constexpr int kOff[4] = {rot_off(0), rot_off(1), rot_off(2), rot_off(3)};  // element of f[i]: g + 32 t + kOff[i]
   // units: 64 codes = elements [0, 64) or [64, 128) of the block (t < 2 or t >= 2);
   // 32 codes (int8) = the 32 elements of one t
   constexpr int kGroups = UT::kCodes == 64 ? 2 : 4;
@@ -1118,7 +1087,7 @@ void gemv_mma_mixed(const MmaArgs& a, int grid, int threads, int M, cudaStream_t
 
 static bool gemv_fused_path(int bits, int N, int K, int M) {
   Plan p;
-  return M == 1 && bits != 0 && make_plan(bits, N, K, p);
+  return M == 1 && bits != 0 && (gemv_imma_fits(bits, N, K, M) || make_plan(bits, N, K, p));
 }
 
 // Workspace of the tensor-core path: rotated x, its group sums, the row-tile
@@ -1153,6 +1122,7 @@ size_t gemv_workspace_bytes(int bits, int N, int K, int M) {
 qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half* zeros,
                         const uint32_t* sign_bits, const __half* x, __half* y, int M,
                         void* workspace, cudaStream_t s) {
+  if (gemv_imma_fits(v.bits, v.N, v.K, M)) return launch_gemv_imma(v, scales, zeros, sign_bits, x, y, s);
   if (gemv_fused_path(v.bits, v.N, v.K, M)) {
     Args a;
     if (make_plan(v.bits, v.N, v.K, a.p)) {
@@ -1207,6 +1177,10 @@ qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half*
 
 void gemv_plan_info(int bits, int N, int K, int M, qlin_gemv_plan_info* info) {
   *info = qlin_gemv_plan_info{};
+  if (gemv_imma_fits(bits, N, K, M)) {
+    gemv_imma_plan_info(bits, N, K, info);
+    return;
+  }
   Plan p;
   if (M == 1 && bits != 0 && make_plan(bits, N, K, p)) {
     info->kernel = 1;

@@ -54,6 +54,13 @@ unsigned take_gemm_error();
 qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half* zeros,
                         const uint32_t* sign_bits, const __half* x, __half* y, int M,
                         void* workspace, cudaStream_t s);
+// The M = 1 integer-tensor-core GEMV (4- and 8-bit codes, a CTA's rows resident
+// in shared memory): whether it takes this shape, and its launch.
+bool gemv_imma_fits(int bits, int N, int K, int M);
+qlin_status launch_gemv_imma(const PackedView& v, const __half* scales, const __half* zeros,
+                             const uint32_t* sign_bits, const __half* x, __half* y, cudaStream_t s);
+void gemv_imma_plan_info(int bits, int N, int K, qlin_gemv_plan_info* info);
+unsigned take_imma_error();
 // Rotation and round-to-nearest quantisation of fp16 weight rows (offline tool).
 qlin_status launch_quantize_rtn(const __half* w, const uint32_t* sign_bits, const uint8_t* block_bits, int bits,
                                 int N, int K, uint8_t* codes, __half* scales, __half* zeros, cudaStream_t s);

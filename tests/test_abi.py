@@ -162,6 +162,14 @@ def test_gemv_plan_invariants(lib):
                 if p["kernel"] == 2:  # very long K: the tensor-core kernel with a workspace
                     assert K // unit > 320 and p["workspace_bytes"] > 0
                     continue
+                if p["kernel"] == 3:  # integer tensor-core kernel: 4/8-bit, a CTA's rows all resident
+                    assert bits in (4, 8) and p["workspace_bytes"] == 0
+                    assert p["threads"] == 32 * (p["consumer_warps"] + 1)
+                    assert p["grid"] == min(148, N) and p["rows_per_cta"] == -(-N // p["grid"])
+                    assert p["rows_per_chunk"] == 16 and p["stages"] == -(-p["rows_per_cta"] // 16) <= 64
+                    assert smem_floor <= p["smem_bytes"] <= smem_limit, (bits, K, N, p)
+                    assert p["rows_per_cta"] * K * bits // 8 < p["smem_bytes"], (bits, K, N, p)
+                    continue
                 U, NW, UW = K // unit, p["consumer_warps"], p["units_per_warp"]
                 assert 1 <= NW <= 10 and UW in (1, 2, 4, 8, 16, 32) and (NW - 1) * UW < U <= NW * UW
                 assert p["threads"] == 32 * (NW + 1)
