@@ -158,6 +158,30 @@ def draw_activation(M: int, K: int, *, seed: int = 0, index: int = 0, device="cp
     return Activation(x, sb.to(torch.int32))
 
 
+CALIB_SEQUENCES = 128
+CALIB_TOKENS = 16
+CALIB_HEAVY_SHARE = 0.01
+CALIB_HEAVY_FACTOR = 8.0
+CALIB_RANK = 8
+
+
+def draw_calibration(K: int, *, seed: int = 0, index: int = 0, n: int = CALIB_SEQUENCES * CALIB_TOKENS,
+                     device="cpu") -> torch.Tensor:
+    """Synthetic calibration inputs of a layer, x [n, K] fp32 (the stand-in for
+    128 calibration sequences): N(0, 1) plus a shared rank-8 component (so the
+    channels correlate), with exactly round(1 % * K) channels, chosen without
+    replacement, scaled by 8 (activation outlier channels)."""
+    g = _gen(device, seed, _STREAM_ACT, 1000 + index)
+    x = torch.randn(n, K, generator=g, device=device, dtype=torch.float32)
+    basis = torch.randn(CALIB_RANK, K, generator=g, device=device, dtype=torch.float32)
+    coef = torch.randn(n, CALIB_RANK, generator=g, device=device, dtype=torch.float32)
+    x += coef @ basis
+    heavy = torch.randperm(K, generator=_gen("cpu", seed, _STREAM_OUTLIERS, 1000 + index))[
+        :int(math.floor(CALIB_HEAVY_SHARE * K + 0.5))]
+    x[:, heavy.to(device)] *= CALIB_HEAVY_FACTOR
+    return x
+
+
 # ---------------------------------------------------------------------------
 # Named workloads
 # ---------------------------------------------------------------------------

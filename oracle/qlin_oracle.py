@@ -26,6 +26,18 @@ What it computes, in the plainest form that the pages support
   Dense 128x128 products, not a butterfly.
 * ``linear64`` -- the fp64 matmul of the rotated activations with the fp64
   dequantised weight.
+* ``hessian64`` / ``hessian_inverse_factor`` / ``gptq_columns32`` / ``gptq32`` /
+  ``quantize_gptq`` -- GPTQ error compensation ("24B0978-Week02-Track2-40-
+  Submission01", section "Recipe": RHT + GPTQ 6-bit g128 from a calibration
+  Hessian of 128 sequences, the compensation run in the rotated basis;
+  "24B0908-Week03-Track1-40-Submission01": GPTQ int3 g128 on the MLP; the
+  Hessian is H = 2 X^T X over the calibration inputs, as the SparseGPT page
+  "24B0908-Week02-Track1-40-Submission01" writes it).  The pages name the
+  method, not its steps; these follow the published column-by-column form:
+  columns in order, each group's grid taken by round-to-nearest from the
+  weights as they stand when the group starts, each column's quantisation
+  error divided by the diagonal of the upper Cholesky factor U of the damped
+  inverse Hessian and subtracted, times U's row, from the later columns.
 * ``rotate_weight32`` / ``rtn32`` / ``quantize_rtn`` -- the offline weight side:
   each weight row rotated with the activations' signs and H / sqrt(128) (the
   weight side of the rotation is folded in offline, "24B0978-Week01-Track2_20-
@@ -45,6 +57,10 @@ Readings where the pages leave a step open (the library documents the same readi
 * Code bits above the width are ignored by ``pack``.
 * Round-to-nearest quantisation works per group in fp32 with the min/max
   affine form above; a zero minimum counts as +0 (so z is -0).
+* GPTQ: damping 1 % of the mean Hessian diagonal; natural column order; the
+  working weights, the factor U and every update in fp32, each product and
+  difference rounded on its own (no fused multiply-add), updates applied to
+  each later column one source column at a time in column order.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 against closed forms, brute force, exact rational arithmetic or a library
@@ -250,6 +266,86 @@ def rtn32(wr: np.ndarray, bits: int | None = None, block_bits=None):
 def quantize_rtn(w: np.ndarray, sign_bits: np.ndarray, bits: int | None = None, block_bits=None):
     """The offline weight side: ``rtn32(rotate_weight32(w))``."""
     return rtn32(rotate_weight32(w, sign_bits), bits, block_bits)
+
+
+# --------------------------------------------------------------------------
+# GPTQ: error-compensated quantisation against a calibration Hessian
+# --------------------------------------------------------------------------
+
+def hessian64(x: np.ndarray) -> np.ndarray:
+    """H = 2 X^T X / n for calibration inputs x [n, K] (rows are the inputs the
+    layer sees), in float64."""
+    x = np.asarray(x, dtype=np.float64)
+    return (2.0 / x.shape[0]) * (x.T @ x)
+
+
+def hessian_inverse_factor(H: np.ndarray, damp: float = 0.01) -> np.ndarray:
+    """Upper-triangular U (float64) with U^T U = (H + damp * mean(diag H) * I)^-1:
+    the lower Cholesky factor of the damped inverse, transposed."""
+    H = np.asarray(H, dtype=np.float64)
+    Hd = H + damp * float(np.mean(np.diag(H))) * np.eye(H.shape[0])
+    return np.linalg.cholesky(np.linalg.inv(Hd)).T
+
+
+def gptq_columns32(w: np.ndarray, U: np.ndarray, qmax: np.ndarray, group: int = GROUP):
+    """The GPTQ column loop on fp32 rows w [N, K] with the fp32 factor U [K, K]
+    and the largest code of each row, qmax [N]:
+
+        for each column i in order:
+            at the first column of a group: its grid (s, z) by round-to-nearest
+                from the group's weights as they are now (the ``rtn32`` formulas);
+            q_i   = clip(rint(w_i / s + z), 0, qmax)
+            e_i   = (w_i - s (q_i - z)) / U[i, i]
+            w_j  -= e_i U[i, j]            for every later column j
+
+    every operation an fp32 operation rounded to nearest.  Returns (codes uint8
+    [N, K], scales fp16 [N, K/group], zeros fp16 [N, K/group], e fp32 [N, K])."""
+    W = np.array(w, dtype=np.float32, copy=True)
+    U = np.asarray(U, dtype=np.float32)
+    N, K = W.shape
+    if K % group or U.shape != (K, K):
+        raise ValueError("K must be a multiple of the group and U must be K x K")
+    qmax = np.asarray(qmax, dtype=np.float32).reshape(N)
+    codes = np.zeros((N, K), dtype=np.uint8)
+    s16 = np.zeros((N, K // group), dtype=np.float16)
+    z16 = np.zeros((N, K // group), dtype=np.float16)
+    err = np.zeros((N, K), dtype=np.float32)
+    s32 = z32 = None
+    for i in range(K):
+        g, j = divmod(i, group)
+        if j == 0:
+            blk = W[:, i:i + group]
+            mn = blk.min(axis=1) + np.float32(0.0)
+            mx = blk.max(axis=1)
+            sg = ((mx - mn) / qmax).astype(np.float16)
+            sg = np.where(sg.astype(np.float32) > np.float32(0.0), sg, np.float16(1.0))
+            s32 = sg.astype(np.float32)
+            zg = (-mn / s32).astype(np.float16)
+            z32 = zg.astype(np.float32)
+            s16[:, g], z16[:, g] = sg, zg
+        q = np.clip(np.rint(W[:, i] / s32 + z32), np.float32(0.0), qmax)
+        wq = s32 * (q - z32)
+        e = (W[:, i] - wq) / U[i, i]
+        W[:, i + 1:] -= np.outer(e, U[i, i + 1:])
+        codes[:, i] = q.astype(np.uint8)
+        err[:, i] = e
+    return codes, s16, z16, err
+
+
+def gptq32(w: np.ndarray, U: np.ndarray, bits: int | None = None, block_bits=None):
+    """GPTQ of fp32 rows w [N, K] in groups of 128 with each row's width (uniform
+    ``bits`` or per 64-row block); returns (codes, scales, zeros) like ``rtn32``."""
+    w = np.asarray(w, dtype=np.float32)
+    qmax = np.float32(2.0) ** row_widths(w.shape[0], bits, block_bits).astype(np.float32) - np.float32(1.0)
+    codes, s16, z16, _ = gptq_columns32(w, U, qmax, GROUP)
+    return codes, s16, z16
+
+
+def quantize_gptq(w: np.ndarray, sign_bits: np.ndarray, U: np.ndarray, bits: int | None = None, block_bits=None):
+    """The offline weight side with error compensation: ``gptq32`` of the rotated
+    rows ``rotate_weight32(w)``; U is the factor of the Hessian of the rotated
+    activations (the compensation runs in the rotated basis)."""
+    return gptq32(rotate_weight32(w, sign_bits), U, bits, block_bits)
 
 
 # --------------------------------------------------------------------------
