@@ -162,6 +162,26 @@ qlin_status qlin_quantize_rtn(const qlin_desc* d, const uint16_t* w, const uint3
                              reinterpret_cast<cudaStream_t>(st));
 }
 
+size_t qlin_gptq_workspace_bytes(const qlin_desc* d) {
+  return check_desc(d) == QLIN_OK ? gptq_workspace_bytes(d->N, d->K) : 0;
+}
+
+qlin_status qlin_quantize_gptq(const qlin_desc* d, const uint16_t* w, const uint32_t* sign_bits,
+                               const float* hinv_factor, uint8_t* codes, uint16_t* scales, uint16_t* zeros,
+                               void* workspace, size_t workspace_bytes, qlin_stream_t st) {
+  qlin_status r = check_desc(d);
+  if (r != QLIN_OK) return r;
+  if (!w || !sign_bits || !hinv_factor || !codes || !scales || !zeros) return QLIN_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(sign_bits) || !aligned16(hinv_factor) || !aligned16(codes) ||
+      !aligned16(scales) || !aligned16(zeros))
+    return QLIN_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < gptq_workspace_bytes(d->N, d->K)) return QLIN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QLIN_ERR_ALIGNMENT;
+  return launch_quantize_gptq(reinterpret_cast<const __half*>(w), sign_bits, hinv_factor, d->block_bits, d->bits,
+                              d->N, d->K, codes, reinterpret_cast<__half*>(scales), reinterpret_cast<__half*>(zeros),
+                              workspace, reinterpret_cast<cudaStream_t>(st));
+}
+
 qlin_status qlin_rht(const uint16_t* x, uint16_t* xr, const uint32_t* sign_bits, int32_t M,
                      int32_t K, qlin_stream_t st) {
   if (!x || !xr || !sign_bits) return QLIN_ERR_INVALID_ARG;

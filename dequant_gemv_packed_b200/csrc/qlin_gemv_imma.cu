@@ -23,10 +23,13 @@
 // from the stored order; the digit planes of x are stored in the same order.
 //
 // CTA layout (one CTA per SM, rows split evenly; all of a CTA's rows resident
-// in shared memory, each row at a stride that makes the fragment loads free
-// of bank conflicts):
-//   * producer warp: one bulk asynchronous copy per weight row (completing on
-//     the barrier of its 16-row tile) and two for the CTA's scales and zeros;
+// in shared memory):
+//   * producer warp: two bulk asynchronous copies per 16-row tile, one per
+//     8-row chunk (completing on the tile's barrier), and two for the CTA's
+//     scales and zeros.  The tile's second chunk starts 64 bytes (4-bit) or 16
+//     bytes (8-bit) past a 128-byte boundary, and MMA row m takes row m / 2 of
+//     chunk m % 2: the lanes of one fragment-load phase read rows of both
+//     chunks, whose pieces then fall in distinct banks;
 //   * 16 consumer warps: rotate x (one block of 128 per warp at a time, on the
 //     tensor cores: qlin_rot16.cuh), write each group's digit planes and
 //     (xs, xs X) to shared memory, then take (16-row tile, group pair) items
@@ -59,12 +62,16 @@ constexpr int kPlaneLo = 144;                 // the low-digit plane, 16 bytes p
                                               // fragment loads (lanes gl = 0 and 1) fall in distinct banks
 constexpr int kGroupXB = 288;                 // bytes of a group's two planes
 constexpr int kXBatch = 8;                    // x blocks a warp loads before rotating
+constexpr int kInflightTiles = 64;            // producer pacing: tiles in flight per CTA
 
 struct ImmaPlan {
   int G, GP;           // groups per row, group pairs (items per tile)
   int grid, rows_max, T;
-  int row_bytes, stride;
+  int row_bytes;
+  int chunk_b;         // offset of a tile's second 8-row chunk from its first
+  int tile_bytes;      // stride of the tiles in shared memory (a multiple of 128)
   int sz_halves;       // halves per array (scales, zeros) in shared memory
+  int inflight;        // tiles whose copies the producer has in flight at once
   int off_sz, off_xb, off_xc, off_part, off_bar;
   int smem_bytes;
 };
@@ -223,13 +230,16 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
       bulk_g2s(z_raw, a.zeros + al, szb, sz_full);
     }
     for (int r = 0; r < T; ++r) {
-      const int rows = min(16, R - 16 * r);
+      // Pace the stream: at most p.inflight tiles in flight, so that this
+      // CTA's copies do not flood the memory system while the kernel before
+      // it (whose x loads are on the critical path) is still running.
+      if (r >= p.inflight && !mbar_wait(&full[r - p.inflight], 0, &g_imma_error)) imma_fail(0x80u);
+      const int rows = min(16, R - 16 * r), ra = min(8, rows), rb = rows - ra;
+      uint8_t* dst = codes_s + (size_t)r * p.tile_bytes;
+      const uint8_t* src = a.codes + (size_t)(n0 + 16 * r) * p.row_bytes;
       mbar_arrive_expect_tx(&full[r], (uint32_t)rows * (uint32_t)p.row_bytes);
-      for (int i = 0; i < rows; ++i) {
-        const int row = 16 * r + i;
-        bulk_g2s(codes_s + (size_t)row * p.stride, a.codes + (size_t)(n0 + row) * p.row_bytes,
-                 (uint32_t)p.row_bytes, &full[r]);
-      }
+      bulk_g2s(dst, src, (uint32_t)(ra * p.row_bytes), &full[r]);
+      if (rb > 0) bulk_g2s(dst + p.chunk_b, src + (size_t)8 * p.row_bytes, (uint32_t)(rb * p.row_bytes), &full[r]);
     }
     return;
   }
@@ -291,9 +301,13 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
     const uint8_t* b1p = (slot == 1 && has1) ? xb + (size_t)(g0 + 1) * kGroupXB + digit_off : zero32;
     const uint4 b0A = lds128(b0p), b0B = lds128(b0p + 16);
     const uint4 b1A = lds128(b1p), b1B = lds128(b1p + 16);
-    const int ra = min(16 * r + gl, R - 1), rb = min(16 * r + gl + 8, R - 1);
-    const uint8_t* rowa = codes_s + (size_t)ra * p.stride + (kGroupBytes / 4) * t;
-    const uint8_t* rowb = codes_s + (size_t)rb * p.stride + (kGroupBytes / 4) * t;
+    // MMA rows gl and gl + 8: rows gl / 2 and gl / 2 + 4 of chunk gl % 2 of the tile
+    const int ca = 16 * r + 8 * (gl & 1) + (gl >> 1);
+    const int ra = min(ca, R - 1), rb = min(ca + 4, R - 1);  // rows past the share read valid data, stored nowhere
+    const int la = ra - 16 * r, lb = rb - 16 * r;              // rows within the tile: chunk = l / 8
+    const uint8_t* tile = codes_s + (size_t)r * p.tile_bytes + (kGroupBytes / 4) * t;
+    const uint8_t* rowa = tile + (la >> 3) * p.chunk_b + (la & 7) * p.row_bytes;
+    const uint8_t* rowb = tile + (lb >> 3) * p.chunk_b + (lb & 7) * p.row_bytes;
     int dl[4] = {0, 0, 0, 0}, dh[4] = {0, 0, 0, 0};
     group_mma<B>(rowa + g0 * kGroupBytes, rowb + g0 * kGroupBytes, b0A, b0B, dl, dh);
     if (has1) group_mma<B>(rowa + (g0 + 1) * kGroupBytes, rowb + (g0 + 1) * kGroupBytes, b1A, b1B, dl, dh);
@@ -318,8 +332,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
     pa += __shfl_xor_sync(0xffffffffu, pa, 1);  // the pair's two groups (lanes t = 0, 1)
     pb += __shfl_xor_sync(0xffffffffu, pb, 1);
     if (t == 0) {
-      part[pp * Rp + 16 * r + gl] = pa;
-      part[pp * Rp + 16 * r + gl + 8] = pb;
+      part[pp * Rp + ca] = pa;
+      part[pp * Rp + ca + 4] = pb;
     }
     item = __shfl_sync(0xffffffffu, next, 0);
   }
@@ -351,17 +365,23 @@ bool make_imma_plan(int b, int N, int K, ImmaPlan& p) {
   p.T = (p.rows_max + 15) / 16;
   if (p.T > kMaxTiles) return false;
   p.row_bytes = K * b / 8;
-  // Row stride: the lanes of one fragment load phase read 16-byte pieces of two
-  // rows; a stride of 64 (4-bit) or 16 (8-bit) mod 128 puts them in distinct banks.
+  // A tile: chunk A (8 rows) at a 128-byte boundary, chunk B (8 rows) at 64
+  // (4-bit) or 16 (8-bit) bytes mod 128 after it.
   const int want = b == 4 ? 64 : 16;
-  p.stride = p.row_bytes + ((want - p.row_bytes % 128) % 128 + 128) % 128;
-  const int codes = (p.rows_max * p.stride + 127) & ~127;
+  const int a_bytes = 8 * p.row_bytes;
+  p.chunk_b = a_bytes + ((want - a_bytes % 128) % 128 + 128) % 128;
+  p.tile_bytes = (p.chunk_b + 8 * p.row_bytes + 127) & ~127;
+  // the last tile holds only the rows left (at most rows_max - 16 (T - 1))
+  const int last = p.rows_max - 16 * (p.T - 1);
+  const int last_bytes = last <= 8 ? last * p.row_bytes : p.chunk_b + (last - 8) * p.row_bytes;
+  const int codes = ((p.T - 1) * p.tile_bytes + last_bytes + 127) & ~127;
   p.sz_halves = (p.rows_max * p.G + 16 + 7) & ~7;
   p.off_sz = codes;
   p.off_xb = (p.off_sz + 4 * p.sz_halves + 127) & ~127;
   p.off_xc = (p.off_xb + p.G * kGroupXB + 32 + 15) & ~15;
   p.off_part = (p.off_xc + p.G * 8 + 127) & ~127;
   p.off_bar = (p.off_part + p.GP * 16 * p.T * 4 + 127) & ~127;
+  p.inflight = kInflightTiles;
   const int end = p.off_bar + (kMaxTiles + 2) * 8 + 16;
   p.smem_bytes = std::max(end, kMinSmem);
   return end <= kSmemLimit;

@@ -64,6 +64,14 @@ unsigned take_imma_error();
 // Rotation and round-to-nearest quantisation of fp16 weight rows (offline tool).
 qlin_status launch_quantize_rtn(const __half* w, const uint32_t* sign_bits, const uint8_t* block_bits, int bits,
                                 int N, int K, uint8_t* codes, __half* scales, __half* zeros, cudaStream_t s);
+// Rotation of fp16 weight rows into fp32 (the offline tools' first step).
+qlin_status launch_rotate_weight(const __half* w, const uint32_t* sign_bits, int N, int K, float* rotated,
+                                 cudaStream_t s);
+// Rotation and error-compensated quantisation (GPTQ) of fp16 weight rows.
+size_t gptq_workspace_bytes(int N, int K);
+qlin_status launch_quantize_gptq(const __half* w, const uint32_t* sign_bits, const float* U, const uint8_t* block_bits,
+                                 int bits, int N, int K, uint8_t* codes, __half* scales, __half* zeros,
+                                 void* workspace, cudaStream_t s);
 size_t gemm_workspace_bytes(int M, int K);
 qlin_status launch_gemm(const PackedView& v, const __half* scales, const __half* zeros,
                         const uint32_t* sign_bits, const __half* x, __half* y, int M,

@@ -32,9 +32,13 @@ constexpr int kWarpsPerBlock = 8;
 constexpr int kGroupsPerWarp = 4;
 
 // Rows [0, N) of the arguments (already offset to the first row), all of width b.
+// kRotateOnly: write the rotated rows (fp32) to `rotated` and stop there (the
+// input of the error-compensated quantiser).
+template <bool kRotateOnly>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) quantize_rtn_kernel(
     const __half* __restrict__ w, const uint32_t* __restrict__ sign_bits, int b, int N, int K,
-    uint8_t* __restrict__ codes, __half* __restrict__ scales, __half* __restrict__ zeros) {
+    uint8_t* __restrict__ codes, __half* __restrict__ scales, __half* __restrict__ zeros,
+    float* __restrict__ rotated) {
   const int G = K / kGroup;
   const long long total = (long long)N * G;
   const int lane = threadIdx.x & 31, t = lane & 7;
@@ -86,6 +90,14 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) quantize_rtn_kernel(
   float f[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) f[j] = __double2float_rn(__dmul_rn(v[j], inv_sqrt));
+  if constexpr (kRotateOnly) {
+    if (live) {
+      float4* out = reinterpret_cast<float4*>(rotated + base);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[j] = make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]);
+    }
+    return;
+  }
 
   // group minimum and maximum (exact)
   float mn = f[0], mx = f[0];
@@ -138,14 +150,27 @@ qlin_status launch_quantize_rtn(const __half* w, const uint32_t* sign_bits, cons
     const long long per_block = (long long)kWarpsPerBlock * kGroupsPerWarp;
     const long long grid = (items + per_block - 1) / per_block;
     if (grid > 0x7fffffffLL) return QLIN_ERR_SHAPE;
-    quantize_rtn_kernel<<<(unsigned)grid, kWarpsPerBlock * 32, 0, s>>>(
+    quantize_rtn_kernel<false><<<(unsigned)grid, kWarpsPerBlock * 32, 0, s>>>(
         w + (size_t)r0 * K, sign_bits, b, r1 - r0, K, codes + (size_t)r0 * K, scales + (size_t)r0 * G,
-        zeros + (size_t)r0 * G);
+        zeros + (size_t)r0 * G, nullptr);
     const qlin_status st = record_cuda(cudaGetLastError());
     if (st != QLIN_OK) return st;
     r0 = r1;
   }
   return QLIN_OK;
+}
+
+// The rotated rows alone, fp32 [N][K]: w~ = fp32(fp64(1/sqrt(128)) (H diag(d) w))
+// per block of 128, the same values the quantiser above works on.
+qlin_status launch_rotate_weight(const __half* w, const uint32_t* sign_bits, int N, int K, float* rotated,
+                                 cudaStream_t s) {
+  const long long items = (long long)N * (K / kGroup);
+  const long long per_block = (long long)kWarpsPerBlock * kGroupsPerWarp;
+  const long long grid = (items + per_block - 1) / per_block;
+  if (grid > 0x7fffffffLL) return QLIN_ERR_SHAPE;
+  quantize_rtn_kernel<true><<<(unsigned)grid, kWarpsPerBlock * 32, 0, s>>>(w, sign_bits, 8, N, K, nullptr, nullptr,
+                                                                           nullptr, rotated);
+  return record_cuda(cudaGetLastError());
 }
 
 }  // namespace qlin

@@ -23,7 +23,7 @@ EXPORTED = (
     "qlin_status_string", "qlin_last_cuda_error", "qlin_packed_bytes", "qlin_code_bytes", "qlin_pack",
     "qlin_unpack", "qlin_dequant", "qlin_rht", "qlin_gemv_workspace_bytes", "qlin_gemv",
     "qlin_gemm_workspace_bytes", "qlin_gemm", "qlin_device_error", "qlin_gemm_noalloc", "qlin_set_overlap",
-    "qlin_quantize_rtn", "qlin_gemv_plan",
+    "qlin_quantize_rtn", "qlin_gemv_plan", "qlin_gptq_workspace_bytes", "qlin_quantize_gptq",
 )
 
 
@@ -85,6 +85,9 @@ def lib() -> ctypes.CDLL:
     L.qlin_dequant.argtypes, L.qlin_dequant.restype = [vp, vp, vp, vp, vp, vp], ctypes.c_int
     L.qlin_rht.argtypes, L.qlin_rht.restype = [vp, vp, vp, i32, i32, vp], ctypes.c_int
     L.qlin_quantize_rtn.argtypes, L.qlin_quantize_rtn.restype = [vp, vp, vp, vp, vp, vp, vp], ctypes.c_int
+    L.qlin_gptq_workspace_bytes.argtypes, L.qlin_gptq_workspace_bytes.restype = [vp], sz
+    L.qlin_quantize_gptq.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.qlin_quantize_gptq.restype = ctypes.c_int
     L.qlin_gemv_plan.argtypes, L.qlin_gemv_plan.restype = [vp, i32, vp], ctypes.c_int
     L.qlin_gemv_workspace_bytes.argtypes, L.qlin_gemv_workspace_bytes.restype = [vp, i32], sz
     L.qlin_gemm_workspace_bytes.argtypes, L.qlin_gemm_workspace_bytes.restype = [vp, i32], sz
@@ -217,6 +220,33 @@ def qlin_quantize_rtn(desc: Desc, w: torch.Tensor, sign_bits: torch.Tensor, code
     _check(lib().qlin_quantize_rtn(desc.ref(), _dev(w, torch.float16, "w"), _dev(sign_bits, torch.int32, "sign_bits"),
                                    _dev(codes, torch.uint8, "codes"), _dev(scales, torch.float16, "scales"),
                                    _dev(zeros, torch.float16, "zeros"), _stream(stream)), "qlin_quantize_rtn")
+    return codes, scales, zeros
+
+
+def qlin_gptq_workspace_bytes(desc: Desc) -> int:
+    return int(lib().qlin_gptq_workspace_bytes(desc.ref()))
+
+
+def qlin_quantize_gptq(desc: Desc, w: torch.Tensor, sign_bits: torch.Tensor, hinv_factor: torch.Tensor,
+                       codes: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None,
+                       zeros: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Rotation and error-compensated (GPTQ) quantisation of fp16 weight rows
+    against the fp32 upper factor of the damped inverse Hessian: (codes, scales, zeros)."""
+    G = desc.K // 128
+    if codes is None:
+        codes = _alloc((desc.N, desc.K), torch.uint8, w)
+    if scales is None:
+        scales = _alloc((desc.N, G), torch.float16, w)
+    if zeros is None:
+        zeros = _alloc((desc.N, G), torch.float16, w)
+    need = qlin_gptq_workspace_bytes(desc)
+    if workspace is None:
+        workspace = _alloc((max(need, 16),), torch.uint8, w)
+    _check(lib().qlin_quantize_gptq(desc.ref(), _dev(w, torch.float16, "w"), _dev(sign_bits, torch.int32, "sign_bits"),
+                                    _dev(hinv_factor, torch.float32, "hinv_factor"), _dev(codes, torch.uint8, "codes"),
+                                    _dev(scales, torch.float16, "scales"), _dev(zeros, torch.float16, "zeros"),
+                                    _dev(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+           "qlin_quantize_gptq")
     return codes, scales, zeros
 
 

@@ -186,6 +186,45 @@ qlin_status qlin_dequant(const qlin_desc* desc, const void* packed, const uint16
 qlin_status qlin_quantize_rtn(const qlin_desc* desc, const uint16_t* w, const uint32_t* sign_bits,
                               uint8_t* codes, uint16_t* scales, uint16_t* zeros, qlin_stream_t stream);
 
+/* Workspace bytes of qlin_quantize_gptq: the rotated rows (fp32 [N][K]), the
+ * quantisation errors of one group of columns (fp32 [N][128]) and the width
+ * table; 0 for an invalid descriptor. */
+size_t qlin_gptq_workspace_bytes(const qlin_desc* desc);
+
+/* Offline weight side with error compensation (GPTQ): rotate each weight row
+ * exactly as qlin_quantize_rtn does, w~ (fp32), then quantise the rotated rows
+ * column by column against a calibration Hessian H, through the upper
+ * triangular factor U of its damped inverse (U^T U = (H + damp I)^-1, the
+ * Hessian of the ROTATED activations; computing H and U is the caller's):
+ *   for each column i in order:
+ *     at the first column of a group of 128: the group's grid by
+ *       round-to-nearest from its weights as they stand now:
+ *       s = fp16_rn((max - min) / (2^b - 1)) (1 if not > 0), z = fp16_rn(-min / s);
+ *     q_i = min(max(rint(w~_i / s + z), 0), 2^b - 1);
+ *     e_i = (w~_i - s (q_i - z)) / U[i][i];
+ *     w~_j = w~_j - e_i U[i][j] for every later column j,
+ * every step an IEEE fp32 operation rounded to nearest (products and
+ * differences rounded separately), each weight updated one source column at a
+ * time in column order: the outputs are a function of (w, sign_bits, U),
+ * bit-exact and deterministic.  With U diagonal nothing propagates and the
+ * result is qlin_quantize_rtn's.
+ *   w           : device fp16 [N][K], the unrotated weight;
+ *   sign_bits   : device uint32 [K/32], the activations' signs;
+ *   hinv_factor : device fp32 [K][K], row-major, upper triangular (only the
+ *                 upper triangle is read), positive diagonal;
+ *   codes       : device uint8 [N][K];  scales, zeros : device fp16 [N][K/128];
+ *   workspace   : device, >= qlin_gptq_workspace_bytes(desc) bytes, overwritten.
+ * Widths: desc->bits or desc->block_bits (copied to the workspace from host
+ * memory, like qlin_pack's table).  No buffer may alias another.
+ * Definition: "24B0978-Week02-Track2-40-Submission01", section "Recipe" (stage
+ * quant_rht_gptq: bits 6, group 128; GPTQ's compensation run in the rotated
+ * basis, calibration Hessian of 128 sequences); "24B0908-Week03-Track1-40-
+ * Submission01" (GPTQ int3, group 128); H = 2 X^T X as written on
+ * "24B0908-Week02-Track1-40-Submission01". */
+qlin_status qlin_quantize_gptq(const qlin_desc* desc, const uint16_t* w, const uint32_t* sign_bits,
+                               const float* hinv_factor, uint8_t* codes, uint16_t* scales, uint16_t* zeros,
+                               void* workspace, size_t workspace_bytes, qlin_stream_t stream);
+
 /* Random Hadamard transform of M rows of K activations.
  *   x  : device fp16 [M][K];  xr : device fp16 [M][K] (may not alias x);
  *   sign_bits : device uint32 [K/32].

@@ -284,7 +284,7 @@ def hessian_inverse_factor(H: np.ndarray, damp: float = 0.01) -> np.ndarray:
     the lower Cholesky factor of the damped inverse, transposed."""
     H = np.asarray(H, dtype=np.float64)
     Hd = H + damp * float(np.mean(np.diag(H))) * np.eye(H.shape[0])
-    return np.linalg.cholesky(np.linalg.inv(Hd)).T
+    return np.ascontiguousarray(np.linalg.cholesky(np.linalg.inv(Hd)).T)
 
 
 def gptq_columns32(w: np.ndarray, U: np.ndarray, qmax: np.ndarray, group: int = GROUP):
