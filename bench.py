@@ -27,6 +27,7 @@ import subprocess
 import sys
 import threading
 import time
+from types import SimpleNamespace
 
 import numpy as np
 import torch
@@ -531,6 +532,71 @@ def cpu_oracle_rate(case: Case, budget_s: float = 12.0, rows_per_step: int | Non
     return gbs, done_rows, t
 
 
+# ------------------------------------------------------------- per-config table
+
+# Every workload of the specification besides the headline one, each timed on
+# its own short region (tens of ms) so that the default run stays short.
+PER_CONFIG = (("tiny", 4000, 20), ("down1", 4000, 20), ("down4", 2000, 20), ("down16", 2000, 20),
+              ("stack", 30, 3), ("stack_fused", 30, 3), ("mid32", 1000, 20), ("prefill256", 1000, 20),
+              ("prefill1024", 400, 10), ("prefill2048", 200, 10), ("quantize", 1000, 20))
+
+
+def workload_config(case, world: int) -> dict:
+    """What the workload is (identical in both arms): shapes, widths, inputs."""
+    bits = getattr(case, "bits", None)
+    return {"workload": case.desc_text, "M": case.M, "K": case.K, "N": case.N, "group": 128,
+            "bits": ("mixed int6/int8" if bits == 0 else bits) if case.kind != "stack" else "int6 + int8 lm_head",
+            "parallelism": f"replicas x{world}",
+            "inputs": "seeded synthetic: weights N(0,0.02) with 0.1% x20 outliers, RTN g128 fp16 scale/zero; "
+                      "activations N(0,1) fp16; random signs"}
+
+
+def roofline_of(case, ms_step: float, peaks: dict) -> dict:
+    """HBM roofline below the ridge point (measured peak FLOP/s over measured HBM
+    bytes/s), tensor roofline above it."""
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if case.kind == "gemm" and case.flops / case.bytes > ridge:
+        achieved = case.flops / (ms_step * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "peak_source": f"{peaks['source']} dense bf16 cuBLAS burst (fp16 nominal ratio 1:1)"}
+    achieved = case.bytes / (ms_step * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} HBM copy bandwidth"}
+
+
+def measure_per_config(stream, peaks: dict, skip: str) -> dict:
+    """One short timed region per workload: us/call, roofline, cuBLAS bf16 of the
+    same shape, and the clocks sampled during that region."""
+    from dequant_gemv_packed_b200 import qlin as Q
+    out = {}
+    for name, steps, warmup in PER_CONFIG:
+        if name == skip:
+            continue
+        case = Case(name)
+        overlap = case.kind in ("gemv", "stack")
+        prev = Q.qlin_set_overlap(overlap)
+        try:
+            ms, clocks = time_steps(case, steps, warmup, None, stream)
+        finally:
+            Q.qlin_set_overlap(prev)
+        ms_step = ms / steps
+        roof = roofline_of(case, ms_step, peaks)
+        entry = {"us_per_call": ms_step * 1e3, "steps": steps, "bound": roof["bound"],
+                 "achieved": roof["achieved"], "unit": roof["unit"], "frac": roof["frac"],
+                 "algorithmic_bytes": case.bytes, "flops": case.flops,
+                 "launches_per_step": case.launches_per_step(), "clocks": clocks,
+                 "launch": "programmatic dependent launch" if overlap else "serial"}
+        cub = time_cublas(case, stream, reps=512)
+        if cub is not None:
+            entry["cublas_bf16_us"] = cub
+            entry["speedup_vs_cublas"] = cub / (ms_step * 1e3)
+        out[name] = entry
+        del case
+        torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------------ main
 
 def run_ours(args):
@@ -558,17 +624,7 @@ def run_ours(args):
     value = whole_job_gbs(case.bytes, args.steps, world, ms)
     per_gpu_gbs = case.bytes / (ms_step * 1e-3) / 1e9
     khash = kernel_source_hash(case.kind)
-    # A GEMM is bound by the tensor cores above the ridge point (measured peak
-    # FLOP/s over measured HBM bytes/s), by HBM below it (mid-batch M).
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if case.kind == "gemm" and case.flops / case.bytes > ridge:
-        achieved = case.flops / (ms_step * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"],
-                "peak_source": f"{peaks['source']} dense bf16 cuBLAS burst (fp16 nominal ratio 1:1)"}
-    else:
-        roof = {"bound": "hbm", "achieved": per_gpu_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": per_gpu_gbs / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} HBM copy bandwidth"}
+    roof = roofline_of(case, ms_step, peaks)
     roof["traffic"] = ncu_traffic(args.workload, khash)
     roof["algorithmic_bytes_per_launch"] = case.bytes
     e2e = None if args.no_extras else time_e2e(case, args.steps, args.warmup, stream)
@@ -590,28 +646,33 @@ def run_ours(args):
         gbs_all, rows_all, t_all = rate(case, budget_s=args.cpu_budget / 2, threads=None)
         cpu_all = {"value": gbs_all, "unit": "GB/s", "cores": ncores, "kind": "oracle",
                    "sample": f"{rows_all} of {case.N} weight rows ({what}), {t_all:.1f} s, BLAS on {ncores} threads"}
+    per_config = None
+    if rank == 0 and world == 1 and not args.no_extras and not args.no_per_config:
+        per_config = measure_per_config(stream, peaks, args.workload)
     if rank == 0:
         us = ms_step * 1e3
-        cfg = {"workload": case.desc_text, "M": case.M, "K": case.K, "N": case.N,
-               "group": 128, "copies": case.copies,
-               "l2": f"rotating {case.copies} weight copies ({case.weight_bytes_total / 1e6:.0f} MB > 2x L2)"
-               if case.kind != "stack" else f"stack weights {case.weight_bytes_total / 1e9:.2f} GB > L2",
-               "parallelism": f"replicas x{world}",
-               "accumulate": "fp64 rotation, fp32 quantiser" if case.kind == "quantize" else "fp32",
-               "kernel_hash": khash,
-               "launch": ("CUDA graph, consecutive calls overlapped by programmatic dependent launch "
-                          "(qlin_set_overlap(1))") if overlap else "CUDA graph, serial launches"}
+        cfg = workload_config(case, world)
+        timing = {"copies": case.copies,
+                  "l2": f"rotating {case.copies} weight copies ({case.weight_bytes_total / 1e6:.0f} MB > 2x L2)"
+                  if case.kind != "stack" else f"stack weights {case.weight_bytes_total / 1e9:.2f} GB > L2",
+                  "accumulate": "fp64 rotation, fp32 quantiser" if case.kind == "quantize" else "fp32",
+                  "kernel_hash": khash,
+                  "launch": ("CUDA graph, consecutive calls overlapped by programmatic dependent launch "
+                             "(qlin_set_overlap(1))") if overlap else "CUDA graph, serial launches",
+                  "region": "device spin, start event, K steps from CUDA graphs, end event"}
         out = {"metric": QUANTIZE_METRIC if case.kind == "quantize" else METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
                "warmup": args.warmup, "ms_per_step": ms_step, "us_per_call": us,
                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                "dtype": "f64" if case.kind == "quantize" else "f16", "data": "synthetic", "config": cfg, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-               "gpu_launches": case.launches_per_step() * args.steps, "clocks": clocks}
+               "gpu_launches": case.launches_per_step() * args.steps, "clocks": clocks, "timing": timing}
         if cpu_all is not None:
             out["cpu_baseline_all_cores"] = cpu_all
         if cublas_us is not None:
             out["cublas_bf16"] = {"us_per_call": cublas_us, "speedup": cublas_us / us}
         if no_overlap is not None:
             out["no_overlap"] = no_overlap
+        if per_config is not None:
+            out["per_config"] = per_config
         print(json.dumps(out), flush=True)
     if dist is not None:
         dist.destroy_process_group()
@@ -666,7 +727,8 @@ def run_reference(args):
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": desc, "M": a.x.shape[0], "K": K, "N": N, "group": 128},
+           "config": workload_config(SimpleNamespace(desc_text=desc, M=a.x.shape[0], K=K, N=N, bits=w.bits, kind=kind),
+                                     int(os.environ.get("WORLD_SIZE", "1"))),
            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -701,7 +763,8 @@ def run_reference_quantize(args, desc, p):
     out = {"impl": "reference", "metric": QUANTIZE_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3 / args.steps,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": desc, "K": K, "N": N, "group": 128, "bits": bits},
+           "config": workload_config(SimpleNamespace(desc_text=desc, M=1, K=K, N=N, bits=bits, kind="quantize"),
+                                     int(os.environ.get("WORLD_SIZE", "1"))),
            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -719,7 +782,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-overlap", action="store_true", help="serial launches only (no programmatic dependent launch)")
     ap.add_argument("--no-extras", action="store_true",
-                    help="time the layer only (no e2e, cuBLAS or CPU-baseline legs), e.g. under a profiler")
+                    help="time the layer only (no e2e, cuBLAS, CPU-baseline or per-config legs), e.g. under a profiler")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the per-config table")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

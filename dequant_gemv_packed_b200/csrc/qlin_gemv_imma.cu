@@ -102,6 +102,31 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ uint4 ldsu128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ float ldsh2f(uint32_t addr) {
+  uint16_t h;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h) : "r"(addr));
+  return __half2float(__ushort_as_half(h));
+}
+
+// The partial sums of this lane's rows (tile rows la and la + 4) for its group
+// (lanes t = 0, 1; `valid` false: no group), added over the pair's two groups
+// and stored by lane t = 0 at part[idx] and part[idx + 4].
+__device__ __forceinline__ void store_pair(float* part, int idx, float pa, float pb, bool valid, int t) {
+  if (!valid) pa = pb = 0.f;
+  pa += __shfl_xor_sync(0xffffffffu, pa, 1);
+  pb += __shfl_xor_sync(0xffffffffu, pb, 1);
+  if (t == 0) {
+    part[idx] = pa;
+    part[idx + 4] = pb;
+  }
+}
+
 // Where code c (0..127) of a group sits in a digit plane.  Lane t's 32 bytes
 // [32t, 32t + 32) are its B fragments in MMA order.
 //   8-bit: lane t's codes are 32t..32t+31, words in MMA order: as stored.
@@ -148,28 +173,6 @@ __device__ __forceinline__ void prepare_group(uint32_t b0, uint32_t b1, uint32_t
     plane[kPlaneLo + pos] = (uint8_t)lo;
   }
   if (lane == 0) *xc = make_float2(xs, xs * (float)xsum);
-}
-
-// The MMAs of one group of one 16-row tile: rows pa (g) and pb (g + 8) at
-// this lane's slice of the group, B fragments bA (plane bytes 0..15 of the
-// lane) and bB (16..31).
-template <int B>
-__device__ __forceinline__ void group_mma(const uint8_t* pa, const uint8_t* pb, uint4 bA, uint4 bB, int (&dl)[4],
-                                          int (&dh)[4]) {
-  if constexpr (B == 4) {
-    constexpr uint32_t kLo = 0x0F0F0F0Fu, kHi = 0xF0F0F0F0u;
-    const uint4 wa = lds128(pa), wb = lds128(pb);
-    mma_u8s8(dl, wa.x & kLo, wb.x & kLo, wa.y & kLo, wb.y & kLo, bA.x, bA.y);
-    mma_u8s8(dl, wa.z & kLo, wb.z & kLo, wa.w & kLo, wb.w & kLo, bA.z, bA.w);
-    mma_u8s8(dh, wa.x & kHi, wb.x & kHi, wa.y & kHi, wb.y & kHi, bB.x, bB.y);
-    mma_u8s8(dh, wa.z & kHi, wb.z & kHi, wa.w & kHi, wb.w & kHi, bB.z, bB.w);
-  } else {
-    const uint4 wa0 = lds128(pa), wa1 = lds128(pa + 16), wb0 = lds128(pb), wb1 = lds128(pb + 16);
-    mma_u8s8(dl, wa0.x, wb0.x, wa0.y, wb0.y, bA.x, bA.y);
-    mma_u8s8(dl, wa0.z, wb0.z, wa0.w, wb0.w, bA.z, bA.w);
-    mma_u8s8(dl, wa1.x, wb1.x, wa1.y, wb1.y, bB.x, bB.y);
-    mma_u8s8(dl, wa1.z, wb1.z, wa1.w, wb1.w, bB.z, bB.w);
-  }
 }
 
 template <int B>
@@ -246,8 +249,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
 
   // ------------------------------------------------------------- prologue --
   // Blocks g = warp, warp + 16, ...: all of the warp's x loads are issued
-  // before any is used (one memory latency).
-  grid_dependency_wait();
+  // before any is used (one memory latency).  The sign bits (weights side) are
+  // read before the dependency wait, x after it.
   {
     uint32_t h[4];
     h16_fragment(lane, h);
@@ -257,10 +260,15 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
 #pragma unroll
       for (int j = 0; j < kXBatch; ++j) {
         const int blk = min(blk0 + j * kNW, G - 1);
+        sw[j] = rot_sign_bits(a.sign_bits, blk, lane);
+      }
+      if (blk0 == warp) grid_dependency_wait();
+#pragma unroll
+      for (int j = 0; j < kXBatch; ++j) {
+        const int blk = min(blk0 + j * kNW, G - 1);
         const __half* xp = a.x + (size_t)blk * kHadamard + xo;
         xb0[j] = *reinterpret_cast<const uint32_t*>(xp);
         xb1[j] = *reinterpret_cast<const uint32_t*>(xp + 8);
-        sw[j] = rot_sign_bits(a.sign_bits, blk, lane);
       }
       if (blk0 == warp) {
         __syncwarp();
@@ -273,69 +281,130 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
         prepare_group<B>(xb0[j], xb1[j], sw[j], h, lane, xb + (size_t)blk * kGroupXB, xc + blk);
       }
     }
-    if (warp >= G && lane == 0) mbar_arrive(x_issued);  // a warp with no block has nothing to load
+    if (warp >= G) {  // a warp with no block has nothing to load
+      grid_dependency_wait();
+      if (lane == 0) mbar_arrive(x_issued);
+    }
   }
   named_barrier(1, kNW * 32);  // digit planes and (xs, xs X) of every group written
   if (!mbar_wait(sz_full, 0, &g_imma_error)) imma_fail(0x20u);
 
   // ------------------------------------------------------------ main loop --
-  const int sz_off = (int)(((size_t)n0 * G) & 7);  // the CTA's first scale in its aligned copy
+  // Items (group pair pp, tile r) in pair-major order, item = pp T + r; warp w
+  // takes the contiguous range [w I / 16, (w + 1) I / 16), so that it loads a
+  // pair's B fragments and x scalars once for all of its tiles of that pair.
+  // Shared memory is addressed with 32-bit offsets computed once per lane.
   const int I = T * GP;
-  const int slot = gl >> 1;                         // this lane's B column: (slot, digit) = (gl / 2, gl % 2)
-  const int digit_off = (gl & 1) * kPlaneLo + 32 * t;
-  int item = 0;
-  if (lane == 0) item = atomicAdd(counter, 1);
-  item = __shfl_sync(0xffffffffu, item, 0);
-  int cur_tile = -1;
-  while (item < I) {
-    int next = 0;
-    if (lane == 0) next = atomicAdd(counter, 1);
-    const int r = item / GP, pp = item - r * GP;
-    if (r != cur_tile) {
+  const int i0 = (int)(((long long)warp * I) / kNW), i1 = (int)(((long long)(warp + 1) * I) / kNW);
+  const int slot = gl >> 1;  // this lane's B column: (slot, digit) = (gl / 2, gl % 2)
+  const uint32_t xb_lane = smem_addr(xb) + (uint32_t)((gl & 1) * kPlaneLo + 32 * t);
+  const uint32_t zero_u = smem_addr(zero32);
+  const uint32_t code0 = smem_addr(codes_s) + (uint32_t)((kGroupBytes / 4) * t);
+  // MMA rows gl and gl + 8 are rows la and la + 4 of chunk gl % 2 of a tile
+  const int la = 8 * (gl & 1) + (gl >> 1);
+  const uint32_t lane_row = (uint32_t)((gl & 1) * p.chunk_b + (gl >> 1) * p.row_bytes);
+  const uint32_t row4 = 4u * (uint32_t)p.row_bytes;
+  const uint32_t s_u = smem_addr(s_raw), z_u = smem_addr(z_raw);
+  const int sz_off = (int)(((size_t)n0 * G) & 7);  // the CTA's first scale in its aligned copy
+  int pp = i0 / T, r = i0 - pp * T;
+  int cur_pp = -1;
+  unsigned long long waited = 0ull;
+  uint4 b0A = {}, b0B = {}, b1A = {}, b1B = {};
+  float2 xv = make_float2(0.f, 0.f);
+  bool has1 = false;
+  int gq = 0;
+  for (int it = i0; it < i1; ++it) {
+    if (pp != cur_pp) {  // warp-uniform: a new pair
+      cur_pp = pp;
+      const int g0 = 2 * pp;
+      has1 = g0 + 1 < G;
+      const uint32_t b0 = slot == 0 ? xb_lane + (uint32_t)(g0 * kGroupXB) : zero_u;
+      const uint32_t b1 = (slot == 1 && has1) ? xb_lane + (uint32_t)((g0 + 1) * kGroupXB) : zero_u;
+      b0A = ldsu128(b0);
+      b0B = ldsu128(b0 + 16);
+      b1A = ldsu128(b1);
+      b1B = ldsu128(b1 + 16);
+      gq = (t == 1 && has1) ? g0 + 1 : g0;  // lanes t = 0, 1: group g0 + t
+      xv = xc[gq];
+    }
+    if (!((waited >> r) & 1ull)) {  // warp-uniform
       if (!mbar_wait_poll(&full[r], 0, &g_imma_error)) imma_fail(0x10u);
-      cur_tile = r;
+      waited |= 1ull << r;
     }
-    const int g0 = 2 * pp;
-    const bool has1 = g0 + 1 < G;  // warp-uniform
-    const uint8_t* b0p = slot == 0 ? xb + (size_t)g0 * kGroupXB + digit_off : zero32;
-    const uint8_t* b1p = (slot == 1 && has1) ? xb + (size_t)(g0 + 1) * kGroupXB + digit_off : zero32;
-    const uint4 b0A = lds128(b0p), b0B = lds128(b0p + 16);
-    const uint4 b1A = lds128(b1p), b1B = lds128(b1p + 16);
-    // MMA rows gl and gl + 8: rows gl / 2 and gl / 2 + 4 of chunk gl % 2 of the tile
-    const int ca = 16 * r + 8 * (gl & 1) + (gl >> 1);
-    const int ra = min(ca, R - 1), rb = min(ca + 4, R - 1);  // rows past the share read valid data, stored nowhere
-    const int la = ra - 16 * r, lb = rb - 16 * r;              // rows within the tile: chunk = l / 8
-    const uint8_t* tile = codes_s + (size_t)r * p.tile_bytes + (kGroupBytes / 4) * t;
-    const uint8_t* rowa = tile + (la >> 3) * p.chunk_b + (la & 7) * p.row_bytes;
-    const uint8_t* rowb = tile + (lb >> 3) * p.chunk_b + (lb & 7) * p.row_bytes;
+    // this lane's two rows (in the last tile, rows past the share read the last row)
+    const uint32_t tile_u = code0 + (uint32_t)r * (uint32_t)p.tile_bytes;
+    uint32_t ra_u = tile_u + lane_row, rb_u = ra_u + row4;
+    int ra = 16 * r + la, rb = ra + 4;
+    if (rb > R - 1) {
+      const int lr = R - 1 - 16 * r;
+      const uint32_t last = tile_u + (uint32_t)((lr >> 3) * p.chunk_b + (lr & 7) * p.row_bytes);
+      if (ra > R - 1) {
+        ra = R - 1;
+        ra_u = last;
+      }
+      rb = R - 1;
+      rb_u = last;
+    }
+    const uint32_t g0b = (uint32_t)(2 * pp * kGroupBytes);
     int dl[4] = {0, 0, 0, 0}, dh[4] = {0, 0, 0, 0};
-    group_mma<B>(rowa + g0 * kGroupBytes, rowb + g0 * kGroupBytes, b0A, b0B, dl, dh);
-    if (has1) group_mma<B>(rowa + (g0 + 1) * kGroupBytes, rowb + (g0 + 1) * kGroupBytes, b1A, b1B, dl, dh);
-    // lane (gl, t < 2): rows ra, rb of group g0 + t; columns (2t: high digit, 2t + 1: low digit)
-    int Sa, Sb;
     if constexpr (B == 4) {
-      Sa = ((dl[0] + (dh[0] >> 4)) << 8) + (dl[1] + (dh[1] >> 4));
-      Sb = ((dl[2] + (dh[2] >> 4)) << 8) + (dl[3] + (dh[3] >> 4));
+      const uint4 wa0 = ldsu128(ra_u + g0b), wb0 = ldsu128(rb_u + g0b);
+      uint4 wa1 = {}, wb1 = {};
+      if (has1) {
+        wa1 = ldsu128(ra_u + g0b + kGroupBytes);
+        wb1 = ldsu128(rb_u + g0b + kGroupBytes);
+      }
+      const float sa = ldsh2f(s_u + 2u * (uint32_t)(sz_off + ra * G + gq));
+      const float za = ldsh2f(z_u + 2u * (uint32_t)(sz_off + ra * G + gq));
+      const float sb = ldsh2f(s_u + 2u * (uint32_t)(sz_off + rb * G + gq));
+      const float zb = ldsh2f(z_u + 2u * (uint32_t)(sz_off + rb * G + gq));
+      constexpr uint32_t kLo = 0x0F0F0F0Fu, kHi = 0xF0F0F0F0u;
+      mma_u8s8(dl, wa0.x & kLo, wb0.x & kLo, wa0.y & kLo, wb0.y & kLo, b0A.x, b0A.y);
+      mma_u8s8(dh, wa0.x & kHi, wb0.x & kHi, wa0.y & kHi, wb0.y & kHi, b0B.x, b0B.y);
+      mma_u8s8(dl, wa0.z & kLo, wb0.z & kLo, wa0.w & kLo, wb0.w & kLo, b0A.z, b0A.w);
+      mma_u8s8(dh, wa0.z & kHi, wb0.z & kHi, wa0.w & kHi, wb0.w & kHi, b0B.z, b0B.w);
+      if (has1) {
+        mma_u8s8(dl, wa1.x & kLo, wb1.x & kLo, wa1.y & kLo, wb1.y & kLo, b1A.x, b1A.y);
+        mma_u8s8(dh, wa1.x & kHi, wb1.x & kHi, wa1.y & kHi, wb1.y & kHi, b1B.x, b1B.y);
+        mma_u8s8(dl, wa1.z & kLo, wb1.z & kLo, wa1.w & kLo, wb1.w & kLo, b1A.z, b1A.w);
+        mma_u8s8(dh, wa1.z & kHi, wb1.z & kHi, wa1.w & kHi, wb1.w & kHi, b1B.z, b1B.w);
+      }
+      // lane (gl, t < 2): rows ra, rb of group g0 + t; columns 2t (high digit), 2t + 1 (low digit)
+      const int Sa = ((dl[0] + (dh[0] >> 4)) << 8) + (dl[1] + (dh[1] >> 4));
+      const int Sb = ((dl[2] + (dh[2] >> 4)) << 8) + (dl[3] + (dh[3] >> 4));
+      store_pair(part, pp * Rp + 16 * r + la, sa * fmaf(-za, xv.y, xv.x * (float)Sa),
+                 sb * fmaf(-zb, xv.y, xv.x * (float)Sb), t == 0 || (t == 1 && has1), t);
     } else {
-      Sa = (dl[0] << 8) + dl[1];
-      Sb = (dl[2] << 8) + dl[3];
+      const float sa = ldsh2f(s_u + 2u * (uint32_t)(sz_off + ra * G + gq));
+      const float za = ldsh2f(z_u + 2u * (uint32_t)(sz_off + ra * G + gq));
+      const float sb = ldsh2f(s_u + 2u * (uint32_t)(sz_off + rb * G + gq));
+      const float zb = ldsh2f(z_u + 2u * (uint32_t)(sz_off + rb * G + gq));
+      {
+        const uint4 wa0 = ldsu128(ra_u + g0b), wa1 = ldsu128(ra_u + g0b + 16);
+        const uint4 wb0 = ldsu128(rb_u + g0b), wb1 = ldsu128(rb_u + g0b + 16);
+        mma_u8s8(dl, wa0.x, wb0.x, wa0.y, wb0.y, b0A.x, b0A.y);
+        mma_u8s8(dh, wa0.z, wb0.z, wa0.w, wb0.w, b0A.z, b0A.w);
+        mma_u8s8(dl, wa1.x, wb1.x, wa1.y, wb1.y, b0B.x, b0B.y);
+        mma_u8s8(dh, wa1.z, wb1.z, wa1.w, wb1.w, b0B.z, b0B.w);
+      }
+      if (has1) {
+        const uint4 wa2 = ldsu128(ra_u + g0b + kGroupBytes), wa3 = ldsu128(ra_u + g0b + kGroupBytes + 16);
+        const uint4 wb2 = ldsu128(rb_u + g0b + kGroupBytes), wb3 = ldsu128(rb_u + g0b + kGroupBytes + 16);
+        mma_u8s8(dl, wa2.x, wb2.x, wa2.y, wb2.y, b1A.x, b1A.y);
+        mma_u8s8(dh, wa2.z, wb2.z, wa2.w, wb2.w, b1A.z, b1A.w);
+        mma_u8s8(dl, wa3.x, wb3.x, wa3.y, wb3.y, b1B.x, b1B.y);
+        mma_u8s8(dh, wa3.z, wb3.z, wa3.w, wb3.w, b1B.z, b1B.w);
+      }
+      // two accumulators for latency only: both hold plain sums
+      const int Sa = ((dl[0] + dh[0]) << 8) + (dl[1] + dh[1]);
+      const int Sb = ((dl[2] + dh[2]) << 8) + (dl[3] + dh[3]);
+      store_pair(part, pp * Rp + 16 * r + la, sa * fmaf(-za, xv.y, xv.x * (float)Sa),
+                 sb * fmaf(-zb, xv.y, xv.x * (float)Sb), t == 0 || (t == 1 && has1), t);
     }
-    const bool valid = t == 0 || (t == 1 && has1);
-    const int g = valid ? g0 + t : g0;
-    const float2 xv = xc[g];
-    const int qa = sz_off + ra * G + g, qb = sz_off + rb * G + g;
-    const float sa = __half2float(s_raw[qa]), za = __half2float(z_raw[qa]);
-    const float sb = __half2float(s_raw[qb]), zb = __half2float(z_raw[qb]);
-    float pa = sa * fmaf(-za, xv.y, xv.x * (float)Sa);
-    float pb = sb * fmaf(-zb, xv.y, xv.x * (float)Sb);
-    if (!valid) pa = pb = 0.f;
-    pa += __shfl_xor_sync(0xffffffffu, pa, 1);  // the pair's two groups (lanes t = 0, 1)
-    pb += __shfl_xor_sync(0xffffffffu, pb, 1);
-    if (t == 0) {
-      part[pp * Rp + ca] = pa;
-      part[pp * Rp + ca + 4] = pb;
+    if (++r == T) {
+      r = 0;
+      ++pp;
     }
-    item = __shfl_sync(0xffffffffu, next, 0);
   }
   named_barrier(1, kNW * 32);
 

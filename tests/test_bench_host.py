@@ -68,3 +68,20 @@ def test_reference_arm_json_line_on_cpu():
     assert line["impl"] == "reference" and line["value"] > 0 and line["steps"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_reference_config_is_the_workload_config():
+    """Both arms print the same `config`: the workload (shapes, widths, inputs),
+    not how it was timed (that is `timing` in our arm's line)."""
+    from types import SimpleNamespace
+    env = dict(os.environ, QLIN_REFERENCE_BUDGET_S="2")
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
+                          "--steps", "2", "--warmup", "3"], cwd=ROOT, env=env, capture_output=True,
+                         text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    desc = bench.WORKLOADS["tiny"][0]
+    ours = bench.workload_config(SimpleNamespace(desc_text=desc, M=1, K=256, N=512, bits=4, kind="gemv"), 1)
+    assert line["config"] == ours
+    names = {name for name, _, _ in bench.PER_CONFIG}
+    assert names <= set(bench.WORKLOADS) and "gateup" not in names
