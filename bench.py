@@ -80,7 +80,8 @@ def measured_peaks():
 
 
 # The .cu file that defines each workload kind's dominant kernel.
-KERNEL_FILE = {"gemv": "qlin_gemv.cu", "stack": "qlin_gemv.cu", "gemm": "qlin_gemm.cu", "quantize": "qlin_quant.cu"}
+KERNEL_FILE = {"gemv": ("qlin_gemv.cu", "qlin_gemv_imma.cu"), "stack": ("qlin_gemv.cu", "qlin_gemv_imma.cu"),
+               "gemm": ("qlin_gemm.cu",), "quantize": ("qlin_quant.cu",), "gptq": ("qlin_gptq.cu", "qlin_quant.cu")}
 QUANTIZE_METRIC = "µs/call and achieved HBM GB/s (fraction of ~8 TB/s) of the offline weight rotation + RTN quantisation"
 
 
@@ -91,7 +92,7 @@ def kernel_source_hash(kind: str = None) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dequant_gemv_packed_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cuh", ".h")) or (f.endswith(".cu") and (kind is None or f == KERNEL_FILE[kind])):
+        if f.endswith((".cuh", ".h")) or (f.endswith(".cu") and (kind is None or f in KERNEL_FILE[kind])):
             h.update(f.encode())
             h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]

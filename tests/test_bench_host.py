@@ -15,8 +15,9 @@ def test_workload_tables_cover_every_kind():
     kinds = {kind for _, kind, _ in bench.WORKLOADS.values()}
     assert kinds <= set(bench.DEFAULT_STEPS) and kinds <= set(bench.KERNEL_FILE)
     csrc = os.path.join(ROOT, "dequant_gemv_packed_b200", "csrc")
-    for f in bench.KERNEL_FILE.values():
-        assert os.path.exists(os.path.join(csrc, f)), f
+    for files in bench.KERNEL_FILE.values():
+        for f in files:
+            assert os.path.exists(os.path.join(csrc, f)), f
 
 
 def test_source_hash_follows_the_kernel_file(tmp_path, monkeypatch):
