@@ -241,9 +241,9 @@ size_t qlin_gemm_workspace_bytes(const qlin_desc* d, int32_t M) {
 
 qlin_status qlin_device_error(uint32_t* code) {
   if (!code) return QLIN_ERR_INVALID_ARG;
-  const unsigned a = take_gemv_error(), b = take_gemm_error(), c = take_imma_error();
-  if (a == ~0u || b == ~0u || c == ~0u) return QLIN_ERR_CUDA;
-  *code = a | c | (b << 8);
+  const unsigned a = take_gemv_error(), b = take_gemm_error(), c = take_imma_error(), d = take_tc_error();
+  if (a == ~0u || b == ~0u || c == ~0u || d == ~0u) return QLIN_ERR_CUDA;
+  *code = a | c | (b << 8) | (d << 16);
   return QLIN_OK;
 }
 

@@ -1090,6 +1090,11 @@ static bool gemv_fused_path(int bits, int N, int K, int M) {
   return M == 1 && bits != 0 && (gemv_imma_fits(bits, N, K, M) || make_plan(bits, N, K, p));
 }
 
+// M = 2..16 with one code width: the split-K tensor-core kernel (qlin_gemv_tc.cu).
+static bool gemv_tc_path(int bits, int N, int K, int M) {
+  return bits != 0 && M >= 2 && gemv_tc_fits(bits, N, K, M);
+}
+
 // Workspace of the tensor-core path: rotated x, its group sums, the row-tile
 // counters and the warps' partial sums.
 struct MmaWorkspace {
@@ -1116,6 +1121,7 @@ struct MmaWorkspace {
 size_t gemv_workspace_bytes(int bits, int N, int K, int M) {
   // The fused M = 1 kernel rotates x in its prologue and needs no workspace.
   if (gemv_fused_path(bits, N, K, M)) return 0;
+  if (gemv_tc_path(bits, N, K, M)) return gemv_tc_workspace_bytes(bits, N, K, M);
   return MmaWorkspace(N, K, M).total;
 }
 
@@ -1123,6 +1129,7 @@ qlin_status launch_gemv(const PackedView& v, const __half* scales, const __half*
                         const uint32_t* sign_bits, const __half* x, __half* y, int M,
                         void* workspace, cudaStream_t s) {
   if (gemv_imma_fits(v.bits, v.N, v.K, M)) return launch_gemv_imma(v, scales, zeros, sign_bits, x, y, s);
+  if (gemv_tc_path(v.bits, v.N, v.K, M)) return launch_gemv_tc(v, scales, zeros, sign_bits, x, y, M, workspace, s);
   if (gemv_fused_path(v.bits, v.N, v.K, M)) {
     Args a;
     if (make_plan(v.bits, v.N, v.K, a.p)) {
@@ -1179,6 +1186,10 @@ void gemv_plan_info(int bits, int N, int K, int M, qlin_gemv_plan_info* info) {
   *info = qlin_gemv_plan_info{};
   if (gemv_imma_fits(bits, N, K, M)) {
     gemv_imma_plan_info(bits, N, K, info);
+    return;
+  }
+  if (gemv_tc_path(bits, N, K, M)) {
+    gemv_tc_plan_info(bits, N, K, M, info);
     return;
   }
   Plan p;

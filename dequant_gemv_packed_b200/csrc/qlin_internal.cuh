@@ -61,6 +61,14 @@ qlin_status launch_gemv_imma(const PackedView& v, const __half* scales, const __
                              const uint32_t* sign_bits, const __half* x, __half* y, cudaStream_t s);
 void gemv_imma_plan_info(int bits, int N, int K, qlin_gemv_plan_info* info);
 unsigned take_imma_error();
+// The split-K tensor-core GEMV for M = 1..16 and one code width (x rotated in
+// the kernel; workspace: per-tile counters and slice partial sums).
+bool gemv_tc_fits(int bits, int N, int K, int M);
+size_t gemv_tc_workspace_bytes(int bits, int N, int K, int M);
+qlin_status launch_gemv_tc(const PackedView& v, const __half* scales, const __half* zeros, const uint32_t* sign_bits,
+                           const __half* x, __half* y, int M, void* workspace, cudaStream_t s);
+void gemv_tc_plan_info(int bits, int N, int K, int M, qlin_gemv_plan_info* info);
+unsigned take_tc_error();
 // Rotation and round-to-nearest quantisation of fp16 weight rows (offline tool).
 qlin_status launch_quantize_rtn(const __half* w, const uint32_t* sign_bits, const uint8_t* block_bits, int bits,
                                 int N, int K, uint8_t* codes, __half* scales, __half* zeros, cudaStream_t s);

@@ -242,16 +242,21 @@ qlin_status qlin_rht(const uint16_t* x, uint16_t* xr, const uint32_t* sign_bits,
  * together).  Fields a kernel does not have are 0. */
 typedef struct {
   int32_t kernel;           /* 1: fused M = 1 kernel (uniform widths);
-                               2: rotation kernel + tensor-core kernel          */
+                               2: rotation kernel + tensor-core kernel (mixed
+                                  widths);
+                               3: M = 1 integer tensor-core kernel (4, 8 bits);
+                               4: split-K tensor-core kernel, x rotated in the
+                                  kernel (M = 2..16, one width)                 */
   int32_t grid;             /* CTAs of the main kernel                         */
   int32_t threads;          /* threads per CTA                                 */
   int32_t smem_bytes;       /* dynamic shared memory per CTA                   */
   int32_t consumer_warps;   /* kernel 1: warps that multiply (plus 1 producer) */
   int32_t units_per_warp;   /* kernel 1: runs of 64 codes (8-bit: 32) per warp */
-  int32_t rows_per_cta;     /* kernel 1: the most rows one CTA owns            */
-  int32_t rows_per_chunk;   /* kernel 1: rows one bulk copy brings in          */
-  int32_t stages;           /* kernel 1: shared-memory stages                  */
-  int32_t chunks_in_flight; /* kernel 1: copies of one CTA in flight at once   */
+  int32_t rows_per_cta;     /* kernels 1, 3, 4: the most rows one CTA owns      */
+  int32_t rows_per_chunk;   /* kernels 1, 3, 4: rows one bulk copy brings in    */
+  int32_t stages;           /* kernels 1, 3: shared-memory stages; 4: buffers   */
+  int32_t chunks_in_flight; /* kernels 1, 3: copies of one CTA in flight at
+                               once; 4: 32-row tiles per buffer                 */
   uint64_t workspace_bytes; /* = qlin_gemv_workspace_bytes(desc, M)            */
 } qlin_gemv_plan_info;
 
@@ -342,7 +347,8 @@ qlin_status qlin_gemm_noalloc(const qlin_desc* desc, const void* packed, const u
 
 /* Reads and clears the device-side error word (0 = no error).  Kernels that
  * wait on shared-memory barriers bound every wait; a wait that gives up sets a
- * bit here instead of hanging (the call's output is then invalid).  Synchronous:
+ * bit here instead of hanging (the call's output is then invalid): bits 0-7
+ * the M = 1 GEMV kernels, 8-15 the GEMM, 16-23 the split-K GEMV.  Synchronous:
  * waits for all work already queued on the device. */
 qlin_status qlin_device_error(uint32_t* code);
 
