@@ -110,6 +110,13 @@ struct RotArgs {
 
 __device__ __forceinline__ void tc_fail(unsigned code) { atomicOr(&g_tc_error, code); }
 
+// Device-scope fetch-and-add with acquire and release semantics.
+__device__ __forceinline__ unsigned atomic_add_acq_rel(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
@@ -485,14 +492,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
     float* mine = a.part + ((size_t)tg * S + s) * kC * kTileRows;
 #pragma unroll
     for (int m = 0; m < kC; ++m) mine[m * kTileRows + lane] = v[m];
-    __threadfence();
+    // The warp's stores, then one acquire-release increment of the tile's
+    // counter by lane 0 (release: the stores before it, ordered by the warp
+    // barrier, are visible to whoever acquires the counter after it).
     __syncwarp();
     unsigned prev = 0;
-    if (lane == 0) prev = atomicAdd(a.counters + tg, 1u);
+    if (lane == 0) prev = atomic_add_acq_rel(a.counters + tg, 1u);
     prev = __shfl_sync(0xffffffffu, prev, 0);
     if (prev != (unsigned)(S - 1)) return;
-    __threadfence();
-    // the loads of kSliceBatch slices are in flight at once
+    __syncwarp();  // lane 0's acquire, then every lane's loads
+    // Last slice: the other slices' sums, kSliceBatch slices' loads in flight
+    // at once (slices past S load slice S - 1 again and are weighted 0).
     const float* all = a.part + (size_t)tg * S * kC * kTileRows + lane;
     float sum[kC];
 #pragma unroll
@@ -501,18 +511,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
       float ld[kSliceBatch][kC];
 #pragma unroll
       for (int i = 0; i < kSliceBatch; ++i) {
-        if (s0 + i < S) {
+        const int si = min(s0 + i, S - 1);
 #pragma unroll
-          for (int m = 0; m < kC; ++m) ld[i][m] = __ldcg(all + ((size_t)(s0 + i) * kC + m) * kTileRows);
-        } else {
-#pragma unroll
-          for (int m = 0; m < kC; ++m) ld[i][m] = 0.f;
-        }
+        for (int m = 0; m < kC; ++m) ld[i][m] = __ldcg(all + ((size_t)si * kC + m) * kTileRows);
       }
 #pragma unroll
       for (int i = 0; i < kSliceBatch; ++i)
+        if (s0 + i < S)
 #pragma unroll
-        for (int m = 0; m < kC; ++m) sum[m] += ld[i][m];
+          for (int m = 0; m < kC; ++m) sum[m] += ld[i][m];
     }
     if (n < N)
 #pragma unroll
