@@ -18,6 +18,10 @@
 //   D = fp32 in tensor memory, columns [0, BN).
 // Warp roles: 0 TMA producer, 1 MMA issuer (one thread) and TMEM owner,
 // 4..7 epilogue (TMEM lane quarters 0..3), 8..15 dequantisation.
+// The epilogue hands the accumulator back to the MMA as soon as it has loaded
+// the last columns; it then converts the tile to fp16 into a whole-tile
+// staging buffer and stores it with one TMA store, while the MMA already runs
+// the next tile (three B stages leave room for that buffer).
 // Dequantisation warp 8 + j owns TMEM lane quarter q = j % 4 (weight rows
 // 32q .. 32q+31 of the tile, one per thread) and the stages of parity h = j / 4
 // (codes [64h, 64h + 64) of every 128-code group).  Each thread copies its own
@@ -43,7 +47,7 @@ __device__ unsigned int g_gemm_error;
 
 namespace {
 
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kBK = 64;        // k per stage: 64 fp16 = one 128-byte swizzle row of B
 constexpr int kBMw = 128;      // weight rows per tile (MMA M)
 constexpr int kBNmax = 256;    // activation rows per tile (MMA N)
@@ -59,7 +63,7 @@ constexpr int kRing = 3;       // 128-code groups in flight per dequantisation t
 constexpr int kSms = 148;
 constexpr int kSlot = 80;      // bytes per thread per group: piece at 0, scale/zero pairs at 64/68 (stride 5 x 16 B: no bank conflicts)
 constexpr int kRingBytes = kRing * kDeqThreads * kSlot;   // 80 KB
-constexpr int kStageOut = 128 * kBMw * 2;                // Y staging: up to 128 activation rows x 128 weight rows, fp16
+constexpr int kStageOut = kBNmax * kBMw * 2;             // Y staging: a whole tile, up to 256 activation rows x 128 weight rows, fp16
 constexpr int kSmemBytes = kStages * kBStage + kRingBytes + kStageOut + 1024 /*barriers*/ + 1024 /*align*/;
 
 struct GemmArgs {
@@ -78,7 +82,7 @@ struct GemmArgs {
   float* partials;   // [P][part_cols][128]
   int part_cols;     // BN rounded up to the 32 columns one TMEM load covers
   int tma_store;     // Y written by TMA tensor stores through shared memory (N % 8 == 0)
-  int box_m;         // activation rows per store box: min(BN, 128)
+  int box_m;         // activation rows per store box: BN (one store per tile)
 };
 
 // The (tile, group range) segments one CTA works through, in order.
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* Bs = smem;
   uint8_t* ring = Bs + kStages * kBStage;
-  __half* ystage = reinterpret_cast<__half*>(ring + kRingBytes);  // [box_m][128]
+  __half* ystage = reinterpret_cast<__half*>(ring + kRingBytes);  // [BN][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kRingBytes + kStageOut);
   uint64_t* st_empty = bars;
   uint64_t* a_full = bars + kStages;
@@ -413,6 +417,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int row = 32 * q + lane;
     const long long T = (long long)tiles * (a.v.K / kGroup);
     const int G = a.v.K / kGroup, P = gridDim.x, c = blockIdx.x;
+    // The accumulator is handed back to the MMA as soon as this warp has
+    // loaded its last columns: the rest of the epilogue (partial sums,
+    // conversion, stores) overlaps the next tile's MMAs.
+    auto release_acc = [&]() {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+    };
     int i = 0, t, g0, g1;
     Segments sg;
     sg.init(a);
@@ -428,6 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         for (int c0 = 0; c0 < a.BN; c0 += 32) {
           uint32_t r[32];
           tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCol + c0), r);
+          if (c0 + 32 >= a.BN) release_acc();
 #pragma unroll
           for (int j = 0; j < 32; ++j) dst[(size_t)(c0 + j) * kBMw] = __uint_as_float(r[j]);
         }
@@ -465,6 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         for (int c0 = 0; c0 < a.BN; c0 += 32) {
           uint32_t r[32];
           tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCol + c0), r);
+          if (c0 + 32 >= a.BN) release_acc();
           float acc[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(r[j]);
@@ -474,20 +488,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             for (int j = 0; j < 32; ++j) acc[j] += __ldcg(src + (size_t)j * kBMw);
           }
           if (a.tma_store) {
-            // a box of box_m activation rows: stage it (fp16, [m][n]), then one thread stores it
-            const int cb = c0 % a.box_m;
-            if (cb == 0 && c0 > 0) {  // the previous box of this tile is in flight: wait for its reads
-              if (q == 0 && lane == 0) tma_store_wait_read();
-              named_barrier(3, 128);
-            }
+            // the whole tile is staged (fp16, [m][n]) and stored by one thread
+            // after the last chunk, while the MMA already runs the next tile
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (cb + j < a.box_m) ystage[(cb + j) * kBMw + row] = __float2half_rn(acc[j]);
-            if (cb + 32 >= a.box_m || c0 + 32 >= a.BN) {
-              fence_async_shared();
-              named_barrier(3, 128);
-              if (q == 0 && lane == 0) tma_store_2d(&ymap, ystage, n0, m0 + c0 - cb);
-            }
+            for (int j = 0; j < 32; ++j) ystage[(c0 + j) * kBMw + row] = __float2half_rn(acc[j]);
           } else if (n < a.v.N) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -496,15 +500,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
           }
         }
+        if (a.tma_store) {
+          fence_async_shared();
+          named_barrier(3, 128);
+          if (q == 0 && lane == 0) tma_store_2d(&ymap, ystage, n0, m0);
+        }
         if (c_last > c) {
           named_barrier(3, 128);  // every epilogue warp has read the partials
           if (q == 0 && lane == 0)
             for (int cc = c + 1; cc <= c_last; ++cc) a.flags[cc] = 0u;
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
     }
     if (a.tma_store && q == 0 && lane == 0) tma_store_wait_all();
   } else if (warp >= kDeqWarp0) {
@@ -667,7 +673,7 @@ qlin_status launch_gemm_rotated(const PackedView& v, const __half* scales, const
   if (cr != CUDA_SUCCESS) return record_cuda(cudaErrorInvalidValue);
   // Y [M][N] fp16: tensor stores need rows of a multiple of 16 bytes
   CUtensorMap ymap;
-  a.box_m = std::min(a.BN, 128);
+  a.box_m = a.BN;
   a.tma_store = (v.N % 8 == 0) ? 1 : 0;
   if (a.tma_store) {
     const cuuint64_t ydims[2] = {(cuuint64_t)v.N, (cuuint64_t)M};
