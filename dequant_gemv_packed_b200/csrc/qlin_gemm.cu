@@ -18,10 +18,10 @@
 //   D = fp32 in tensor memory, columns [0, BN).
 // Warp roles: 0 TMA producer, 1 MMA issuer (one thread) and TMEM owner,
 // 4..7 epilogue (TMEM lane quarters 0..3), 8..15 dequantisation.
-// The epilogue hands the accumulator back to the MMA as soon as it has loaded
-// the last columns; it then converts the tile to fp16 into a whole-tile
-// staging buffer and stores it with one TMA store, while the MMA already runs
-// the next tile (three B stages leave room for that buffer).
+// The epilogue converts the tile to fp16 into a whole-tile staging buffer,
+// hands the accumulator back to the MMA, and stores the buffer with one TMA
+// store while the MMA already runs the next tile (three B stages leave room
+// for the buffer).
 // Dequantisation warp 8 + j owns TMEM lane quarter q = j % 4 (weight rows
 // 32q .. 32q+31 of the tile, one per thread) and the stages of parity h = j / 4
 // (codes [64h, 64h + 64) of every 128-code group).  Each thread copies its own
@@ -478,7 +478,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         for (int c0 = 0; c0 < a.BN; c0 += 32) {
           uint32_t r[32];
           tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCol + c0), r);
-          if (c0 + 32 >= a.BN) release_acc();
           float acc[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(r[j]);
@@ -500,6 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
           }
         }
+        release_acc();  // every column of the accumulator has been loaded
         if (a.tma_store) {
           fence_async_shared();
           named_barrier(3, 128);
