@@ -52,6 +52,9 @@ WORKLOADS = {
                     "(2560->19456) fused, each sharing one x, M=1 (145 GEMVs per step)", "stack", dict(fused=True)),
     "quantize": ("offline weight side: rotation (signs + block-128 FWHT, fp64) and RTN int4 g128 quantisation "
                  "of an fp16 weight, K=2560, N=9728", "quantize", dict(N=9728, K=2560, bits=4)),
+    "gptq": ("offline weight side with error compensation: rotation (signs + block-128 FWHT) and GPTQ int6 g128 "
+             "against a synthetic calibration Hessian (damped 1 %), q-proj shape K=2560, N=4096", "gptq",
+             dict(N=4096, K=2560, bits=6)),
     "mid32": ("mid-batch dequant-GEMM: M=32, K=2560, N=9728, mixed int6/int8 64-row blocks, block-128 RHT",
               "gemm", dict(M=32)),
     "prefill256": ("prefill dequant-GEMM: M=256, K=2560, N=9728, mixed int6/int8 64-row blocks, block-128 RHT",
@@ -65,7 +68,11 @@ WORKLOADS = {
 
 # Default timed steps per workload kind: about a second of timed work (a
 # gate/up call is ~5 us, a stack step ~2 ms, a prefill GEMM 40-150 us).
-DEFAULT_STEPS = {"gemv": 100000, "stack": 500, "gemm": 10000, "quantize": 20000}
+DEFAULT_STEPS = {"gemv": 100000, "stack": 500, "gemm": 10000, "quantize": 20000, "gptq": 20}
+
+# fp32 instruction peak of the CUDA cores (nominal unit counts and clock: 148 SMs
+# x 128 fp32 lanes x 1965 MHz), for work that may not fuse multiply and add.
+FP32_ALU_TOPS = 148 * 128 * 1.965e9 / 1e12
 
 
 # --------------------------------------------------------------------------- utils
@@ -80,9 +87,11 @@ def measured_peaks():
 
 
 # The .cu file that defines each workload kind's dominant kernel.
-KERNEL_FILE = {"gemv": ("qlin_gemv.cu", "qlin_gemv_imma.cu"), "stack": ("qlin_gemv.cu", "qlin_gemv_imma.cu"),
+KERNEL_FILE = {"gemv": ("qlin_gemv.cu", "qlin_gemv_imma.cu", "qlin_gemv_tc.cu"),
+               "stack": ("qlin_gemv.cu", "qlin_gemv_imma.cu", "qlin_gemv_tc.cu"),
                "gemm": ("qlin_gemm.cu",), "quantize": ("qlin_quant.cu",), "gptq": ("qlin_gptq.cu", "qlin_quant.cu")}
 QUANTIZE_METRIC = "µs/call and achieved HBM GB/s (fraction of ~8 TB/s) of the offline weight rotation + RTN quantisation"
+GPTQ_METRIC = "µs/call and fp32 TFLOP/s (fraction of the CUDA cores' fp32 instruction rate) of rotation + GPTQ"
 
 
 def kernel_source_hash(kind: str = None) -> str:
@@ -237,6 +246,35 @@ class Case:
             self.host_sample = None
             torch.cuda.synchronize()
             return
+        if kind == "gptq":
+            N, K, bits = p["N"], p["K"], p["bits"]
+            self.M, self.N, self.K, self.bits, self.block_bits = 1, N, K, bits, None
+            self.d = Q.Desc(N, K, bits)
+            self.w = [W.draw_fp16_weight(N, K, device=dev)]
+            a = W.draw_activation(1, K, device=dev)
+            # the inverse-Hessian factor is an input: H = 2 X^T X / n of the
+            # synthetic calibration draw, damped by 1 % of its mean diagonal,
+            # U = chol((H + damp I)^-1)^T (fp64 library routines, then fp32)
+            xc = W.draw_calibration(K, device=dev).double()
+            H = (2.0 / xc.shape[0]) * (xc.T @ xc)
+            H += 0.01 * torch.diagonal(H).mean() * torch.eye(K, dtype=torch.float64, device=dev)
+            self.U = torch.linalg.cholesky(torch.linalg.inv(H)).T.contiguous().float()
+            del xc, H
+            G = K // 128
+            self.bytes = N * K * 2 + N * K + 4 * N * G
+            # algorithmic fp32 operations: every column's error updates every later
+            # column of the row, one multiply and one subtraction each
+            self.flops = N * K * (K - 1)
+            self.copies = 1
+            self.out = [(torch.empty(N, K, dtype=torch.uint8, device=dev),
+                         torch.empty(N, G, dtype=torch.float16, device=dev),
+                         torch.empty(N, G, dtype=torch.float16, device=dev))]
+            self.ws = torch.empty(Q.qlin_gptq_workspace_bytes(self.d), dtype=torch.uint8, device=dev)
+            self.weight_bytes_total = N * K * 2
+            self.sign_bits, self.x = a.sign_bits, a.x
+            self.host_sample = None
+            torch.cuda.synchronize()
+            return
         if kind == "quantize":
             N, K, bits = p["N"], p["K"], p["bits"]
             self.M, self.N, self.K, self.bits, self.block_bits = 1, N, K, bits, None
@@ -291,6 +329,8 @@ class Case:
         from dequant_gemv_packed_b200 import qlin as Q
         if self.kind == "quantize":
             return 1  # uniform width: one launch
+        if self.kind == "gptq":
+            return 2 * (self.K // 128)  # the rotation, then per group a block and (but the last) a trailing kernel
         if self.kind == "stack":
             return sum(Q.kernel_launches_per_call("gemv", l[0], 1) for l in self.layers)
         return Q.kernel_launches_per_call(self.kind, self.d, self.M)
@@ -300,6 +340,10 @@ class Case:
         if self.kind == "quantize":
             c, sc, z = self.out[i % 2]
             Q.qlin_quantize_rtn(self.d, self.w[i % self.copies], self.sign_bits, c, sc, z)
+            return
+        if self.kind == "gptq":
+            c, sc, z = self.out[0]
+            Q.qlin_quantize_gptq(self.d, self.w[0], self.sign_bits, self.U, c, sc, z, self.ws)
             return
         if self.kind == "stack":
             for (d, packed, s, z, sb, x, y, ws) in self.layers:
@@ -369,7 +413,7 @@ def time_steps(case: Case, K: int, W: int, dist, stream, graph_len: int = 1024):
 def time_e2e(case: Case, K: int, W: int, stream):
     """Through the public binding, eager: per step copy x in from pinned host
     memory, run the layer, copy y back to pinned host memory."""
-    if case.kind == "stack":
+    if case.kind in ("stack", "gptq"):
         return None
     if case.kind == "quantize":
         return time_e2e_quantize(case, K, W, stream)
@@ -433,7 +477,7 @@ def time_e2e_quantize(case: Case, K: int, W: int, stream):
 
 def time_cublas(case: Case, stream, reps: int = 2000):
     """bf16 torch.nn.functional.linear (cuBLAS) of the same shape, same rotation."""
-    if case.kind in ("stack", "quantize"):
+    if case.kind in ("stack", "quantize", "gptq"):
         return None
     copies = max(1, math.ceil(2 * L2_BYTES / (case.N * case.K * 2)) + 1)
     ws = [torch.randn(case.N, case.K, device="cuda", dtype=torch.bfloat16) for _ in range(copies)]
@@ -539,7 +583,7 @@ def cpu_oracle_rate(case: Case, budget_s: float = 12.0, rows_per_step: int | Non
 # its own short region (tens of ms) so that the default run stays short.
 PER_CONFIG = (("tiny", 4000, 20), ("down1", 4000, 20), ("down4", 2000, 20), ("down16", 2000, 20),
               ("stack", 30, 3), ("stack_fused", 30, 3), ("mid32", 1000, 20), ("prefill256", 1000, 20),
-              ("prefill1024", 400, 10), ("prefill2048", 200, 10), ("quantize", 1000, 20))
+              ("prefill1024", 400, 10), ("prefill2048", 200, 10), ("quantize", 1000, 20), ("gptq", 5, 3))
 
 
 def workload_config(case, world: int) -> dict:
@@ -556,6 +600,11 @@ def roofline_of(case, ms_step: float, peaks: dict) -> dict:
     """HBM roofline below the ridge point (measured peak FLOP/s over measured HBM
     bytes/s), tensor roofline above it."""
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if case.kind == "gptq":
+        achieved = case.flops / (ms_step * 1e-3) / 1e12
+        return {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TOPS, "unit": "TFLOP/s",
+                "frac": achieved / FP32_ALU_TOPS,
+                "peak_source": "nominal fp32 instruction rate: 148 SMs x 128 lanes x 1965 MHz (no fused multiply-add)"}
     if case.kind == "gemm" and case.flops / case.bytes > ridge:
         achieved = case.flops / (ms_step * 1e-3) / 1e12
         return {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -661,10 +710,15 @@ def run_ours(args):
                   "launch": ("CUDA graph, consecutive calls overlapped by programmatic dependent launch "
                              "(qlin_set_overlap(1))") if overlap else "CUDA graph, serial launches",
                   "region": "device spin, start event, K steps from CUDA graphs, end event"}
-        out = {"metric": QUANTIZE_METRIC if case.kind == "quantize" else METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        metric = {"quantize": QUANTIZE_METRIC, "gptq": GPTQ_METRIC}.get(case.kind, METRIC)
+        if case.kind == "gptq":  # whole-job fp32 operations per second
+            value, unit = world * case.flops * args.steps / (ms * 1e-3) / 1e12, "TFLOP/s"
+        else:
+            unit = "GB/s"
+        out = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
                "warmup": args.warmup, "ms_per_step": ms_step, "us_per_call": us,
                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-               "dtype": "f64" if case.kind == "quantize" else "f16", "data": "synthetic", "config": cfg, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+               "dtype": {"quantize": "f64", "gptq": "f32"}.get(case.kind, "f16"), "data": "synthetic", "config": cfg, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                "gpu_launches": case.launches_per_step() * args.steps, "clocks": clocks, "timing": timing}
         if cpu_all is not None:
             out["cpu_baseline_all_cores"] = cpu_all
@@ -690,6 +744,9 @@ def run_reference(args):
     desc, kind, p = WORKLOADS[args.workload]
     if kind == "stack":
         print(json.dumps({"impl": "reference", "unavailable": "stack workload is not sampled by the CPU oracle arm"}))
+        return
+    if kind == "gptq":
+        print(json.dumps({"impl": "reference", "unavailable": "the GPTQ workload is timed only on the GPU arm"}))
         return
     if kind == "quantize":
         run_reference_quantize(args, desc, p)
