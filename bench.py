@@ -53,8 +53,8 @@ WORKLOADS = {
     "quantize": ("offline weight side: rotation (signs + block-128 FWHT, fp64) and RTN int4 g128 quantisation "
                  "of an fp16 weight, K=2560, N=9728", "quantize", dict(N=9728, K=2560, bits=4)),
     "gptq": ("offline weight side with error compensation: rotation (signs + block-128 FWHT) and GPTQ int6 g128 "
-             "against a synthetic calibration Hessian (damped 1 %), q-proj shape K=2560, N=4096", "gptq",
-             dict(N=4096, K=2560, bits=6)),
+             "against a synthetic calibration Hessian (damped 1 %), gate/up-proj shape K=2560, N=9728", "gptq",
+             dict(N=9728, K=2560, bits=6)),
     "mid32": ("mid-batch dequant-GEMM: M=32, K=2560, N=9728, mixed int6/int8 64-row blocks, block-128 RHT",
               "gemm", dict(M=32)),
     "prefill256": ("prefill dequant-GEMM: M=256, K=2560, N=9728, mixed int6/int8 64-row blocks, block-128 RHT",
@@ -703,8 +703,10 @@ def run_ours(args):
         us = ms_step * 1e3
         cfg = workload_config(case, world)
         timing = {"copies": case.copies,
-                  "l2": f"rotating {case.copies} weight copies ({case.weight_bytes_total / 1e6:.0f} MB > 2x L2)"
-                  if case.kind != "stack" else f"stack weights {case.weight_bytes_total / 1e9:.2f} GB > L2",
+                  "l2": (f"stack weights {case.weight_bytes_total / 1e9:.2f} GB > L2" if case.kind == "stack" else
+                         f"fp16 weight {case.N * case.K * 2 / 1e6:.0f} MB + its fp32 working copy "
+                         f"{case.N * case.K * 4 / 1e6:.0f} MB > L2" if case.kind == "gptq" else
+                         f"rotating {case.copies} weight copies ({case.weight_bytes_total / 1e6:.0f} MB > 2x L2)"),
                   "accumulate": "fp64 rotation, fp32 quantiser" if case.kind == "quantize" else "fp32",
                   "kernel_hash": khash,
                   "launch": ("CUDA graph, consecutive calls overlapped by programmatic dependent launch "
