@@ -97,5 +97,18 @@ def test_shared_workspace_across_shapes():
         assert_close(own[:, torch.as_tensor(rows, device=DEV)], oracle_rows(w, a, rows), f"shape {shapes[i]}")
 
 
+@pytest.mark.parametrize("bits", [3, 4, 6, 8])
+@pytest.mark.parametrize("N,K,M", [(1, 128, 16), (31, 128, 2), (33, 9728, 2), (2560, 128, 9), (4097, 256, 8),
+                                   (9728, 2560, 16), (1024, 9728, 3)])
+def test_edge_shapes(bits, N, K, M):
+    """One group (K = 128, a single slice), one row, a row count just past a
+    tile, very long K with few rows, many rows with short K, and the gate/up
+    shape at M = 16 (sampled rows where the layer is large)."""
+    rows = None if N * K <= (1 << 22) else sample_rows(N, 96, seed=N + K)
+    w, a, d, packed, y = _case(N, K, bits, M, seed=N + K + M, rows=rows)
+    if rows is None:
+        assert_dot_bound(y, w, a, what=f"b{bits} N{N} K{K} M{M}")
+
+
 def test_no_tc_errors():
     assert Q.qlin_device_error() == 0
