@@ -33,11 +33,12 @@
 //     the definition.
 //   * reduction in a fixed order: a warp that covers a whole tile's units of
 //     the slice writes its sums out directly; tiles shared by several warps
-//     are added in warp order; with S > 1 the slices' sums go to the workspace
-//     and the last CTA to finish a tile (an atomic counter, zeroed by a memset
-//     node before the launch: the workspace may hold anything on entry) adds
-//     them in slice order and writes y (fp16).  Results do not depend on
-//     timing.
+//     are added in warp order; with S > 1 the S slices of a row part run as
+//     one thread-block cluster, each CTA keeps its tile sums in its shared
+//     memory, and after a cluster barrier each adds all slices' sums for its
+//     share of the outputs, in slice order, reading the others' shared memory
+//     (distributed shared memory), and writes y (fp16).  No global partial
+//     sums, counters or atomics; results do not depend on timing.
 // With qlin_set_overlap(1) the kernel is a programmatic dependent: codes,
 // scales, zeros and signs are fetched before the wait for the previous
 // kernel; x, the workspace and y are touched after it.
@@ -59,11 +60,14 @@ namespace {
 constexpr int kW = 8;                 // warps per CTA
 constexpr int kThreads = kW * 32;
 constexpr int kTileRows = 32;
-constexpr int kSms = 148;
 constexpr int kSmemMax = 227 * 1024;
 constexpr int kSzBatch = 8;           // (scale, zero) pairs a thread loads ahead of the dependency wait
 constexpr int kXBatch = 8;            // x blocks a warp loads before rotating
-constexpr int kSliceBatch = 4;        // slices whose partial sums one lane loads at once
+constexpr int kMaxCluster = 8;        // K slices of a row part: one portable thread-block cluster
+// Clusters of S CTAs that fit on the GPU at once with one CTA per SM (B200, 148
+// SMs in GPCs of 18 or 20; cudaOccupancyMaxActiveClusters at 160 KB and more
+// of shared memory): the grid never exceeds one wave of clusters.
+constexpr int kClustersAtOnce[kMaxCluster + 1] = {0, 148, 74, 45, 33, 26, 22, 15, 15};
 constexpr uint32_t kMagic = 0x64006400u;  // fp16 1024.0 in both halves
 
 struct TcPlan {
@@ -73,14 +77,13 @@ struct TcPlan {
   int Tc;              // most tiles of a part
   int RT, nbuf;        // tiles per round, code buffers (1: one round)
   int NT;              // n8 tiles of x rows (1: M <= 8, 2: M <= 16)
-  int off_xsum, off_sz, off_red, off_codes, off_bar;
+  int off_xsum, off_sz, off_red, off_cp, off_codes, off_bar;
   int buf_bytes;       // one code buffer
   int smem_bytes;
   int xrot;            // 1: x rotated once per call by rot_tc_kernel into the workspace
-  // workspace: counters [T] at 0, partials [T][S][8 NT][32] at ws_part (S > 1),
-  // then (xrot) x~ in the shared-memory layout [G][NT][8][256 B] at ws_xs and
-  // the group sums [G][16] at ws_xsum
-  size_t ws_part, ws_xs, ws_xsum, ws_total;
+  // workspace (xrot plans only): x~ in the shared-memory layout
+  // [G][NT][8][256 B] at ws_xs and the group sums [G][16] at ws_xsum
+  size_t ws_xs, ws_xsum, ws_total;
 };
 
 struct TcArgs {
@@ -91,8 +94,6 @@ struct TcArgs {
   const uint32_t* sign_bits;
   const __half* x;
   __half* y;
-  uint32_t* counters;  // [T], zeroed before the launch
-  float* part;         // [T][S][8 NT][32]
   const uint8_t* xrot; // xrot plans: x~ of every group in the shared-memory layout
   const float* xsum_g; // xrot plans: [G][16] group sums
   int N, K, M;
@@ -104,17 +105,25 @@ struct RotArgs {
   const uint32_t* sign_bits;
   uint8_t* xrot;       // [G][NT][8][256 B]
   float* xsum_g;       // [G][16]
-  uint32_t* counters;  // zeroed: [nclear]
-  int M, K, G, nclear;
+  int M, K, G;
 };
 
 __device__ __forceinline__ void tc_fail(unsigned code) { atomicOr(&g_tc_error, code); }
 
-// Device-scope fetch-and-add with acquire and release semantics.
-__device__ __forceinline__ unsigned atomic_add_acq_rel(unsigned* p, unsigned v) {
-  unsigned old;
-  asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
+// Barrier of every thread of every CTA of the cluster; shared-memory writes
+// before it are visible to the cluster's loads after it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// fp32 at this CTA's shared address `addr`, read from the same address in the
+// shared memory of cluster CTA `rank`.
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr, uint32_t rank) {
+  uint32_t remote;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
@@ -333,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
   float* xsum = reinterpret_cast<float*>(smem + p.off_xsum);  // [Gs][16]
   uint32_t* sz = reinterpret_cast<uint32_t*>(smem + p.off_sz);  // [RT * 32][Gs] (s, z) fp16 pairs
   float* red = reinterpret_cast<float*>(smem + p.off_red);    // [kW][3][32][8 NT + 1]
+  float* cpart = reinterpret_cast<float*>(smem + p.off_cp);   // S > 1: [RT][8 NT][32] this slice's tile sums
   uint8_t* codes = smem + p.off_codes;                        // [nbuf][RT][32][pitch]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
 
@@ -475,56 +485,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
   float* my_red = red + (size_t)warp * 3 * kTileRows * kRS;
 
   // Emits the slice's sums of tile `tl` (local, round r); lane = row of the
-  // tile, v[m] its sums for x rows m: to y (S = 1), else to the workspace and,
-  // for the last slice to arrive, the sum over slices (in slice order) to y.
-  // Called by one whole warp.  Partials are [tile][slice][m][32 rows]: every
-  // store and load of a warp covers 128 contiguous bytes.
+  // tile, v[m] its sums for x rows m: to y (S = 1), else to this CTA's
+  // shared-memory tile sums, which the cluster adds after the round.  Called
+  // by one whole warp.
   auto emit_tile = [&](int r, int tl, const float (&v)[kC]) {
-    const int tg = t0 + r * p.RT + tl;  // global tile
-    const int n = tg * kTileRows + lane;
     if (S == 1) {
+      const int n = (t0 + r * p.RT + tl) * kTileRows + lane;
       if (n < N)
 #pragma unroll
         for (int m = 0; m < kC; ++m)
           if (m < M) a.y[(size_t)m * N + n] = __float2half_rn(v[m]);
       return;
     }
-    float* mine = a.part + ((size_t)tg * S + s) * kC * kTileRows;
 #pragma unroll
-    for (int m = 0; m < kC; ++m) mine[m * kTileRows + lane] = v[m];
-    // The warp's stores, then one acquire-release increment of the tile's
-    // counter by lane 0 (release: the stores before it, ordered by the warp
-    // barrier, are visible to whoever acquires the counter after it).
-    __syncwarp();
-    unsigned prev = 0;
-    if (lane == 0) prev = atomic_add_acq_rel(a.counters + tg, 1u);
-    prev = __shfl_sync(0xffffffffu, prev, 0);
-    if (prev != (unsigned)(S - 1)) return;
-    __syncwarp();  // lane 0's acquire, then every lane's loads
-    // Last slice: the other slices' sums, kSliceBatch slices' loads in flight
-    // at once (slices past S load slice S - 1 again and are weighted 0).
-    const float* all = a.part + (size_t)tg * S * kC * kTileRows + lane;
-    float sum[kC];
-#pragma unroll
-    for (int m = 0; m < kC; ++m) sum[m] = 0.f;
-    for (int s0 = 0; s0 < S; s0 += kSliceBatch) {
-      float ld[kSliceBatch][kC];
-#pragma unroll
-      for (int i = 0; i < kSliceBatch; ++i) {
-        const int si = min(s0 + i, S - 1);
-#pragma unroll
-        for (int m = 0; m < kC; ++m) ld[i][m] = __ldcg(all + ((size_t)si * kC + m) * kTileRows);
-      }
-#pragma unroll
-      for (int i = 0; i < kSliceBatch; ++i)
-        if (s0 + i < S)
-#pragma unroll
-          for (int m = 0; m < kC; ++m) sum[m] += ld[i][m];
-    }
-    if (n < N)
-#pragma unroll
-      for (int m = 0; m < kC; ++m)
-        if (m < M) a.y[(size_t)m * N + n] = __float2half_rn(sum[m]);
+    for (int m = 0; m < kC; ++m) cpart[((size_t)tl * kC + m) * kTileRows + lane] = v[m];
   };
 
   for (int r = 0; r < rounds; ++r) {
@@ -672,6 +646,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
         emit_tile(r, tl, v);
       }
     }
+    if (S > 1) {
+      // The K slices of this row part are the CTAs of one cluster: after the
+      // barrier every slice's tile sums are visible; CTA s adds, in slice
+      // order, the elements [s E / S, (s + 1) E / S) of the round's E = x rows
+      // x tile rows outputs (m-major: consecutive threads, consecutive rows)
+      // and writes them to y.  The second barrier keeps every CTA's sums in
+      // place until all have been read.
+      cluster_sync();
+      const int Rr = nt_r * kTileRows, E = kC * Rr;
+      const int e0 = (int)(((long long)s * E) / S), e1 = (int)(((long long)(s + 1) * E) / S);
+      const uint32_t cp_u = smem_addr(cpart);
+      for (int e = e0 + tid; e < e1; e += kThreads) {
+        const int m = e / Rr, row = e - m * Rr;
+        const int n = (t0 + r * p.RT) * kTileRows + row;
+        if (m >= M || n >= N) continue;
+        const int tl = row / kTileRows, lr = row - tl * kTileRows;
+        const uint32_t addr = cp_u + 4u * (uint32_t)(((tl * kC) + m) * kTileRows + lr);
+        float v = 0.f;
+        for (int ss = 0; ss < S; ++ss) v += ld_cluster_f32(addr, (uint32_t)ss);
+        a.y[(size_t)m * N + n] = __float2half_rn(v);
+      }
+      cluster_sync();
+    }
     __syncthreads();  // the round's codes and segments are no longer read
     if (tid == 0 && r + p.nbuf < rounds) issue_round(r + p.nbuf);
   }
@@ -681,8 +678,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
 // 8 NT, writes group g of row m of x~ (rows m >= M: zeros) as one 256-byte
 // row of gemv_tc_kernel's shared-memory layout (pairs in MMA order, chunks
 // XOR-swizzled by row) and the group's sum; the GEMV's CTAs then copy their
-// slices with one bulk copy each.  Also zeroes the GEMV's tile counters, after
-// the wait for the previous kernel (which may be a GEMV using them).
+// slices with one bulk copy each.  It writes the workspace only after the wait
+// for the previous kernel (which may be a GEMV still reading it).
 template <int B, int NT>
 __global__ void __launch_bounds__(kThreads) rot_tc_kernel(const __grid_constant__ RotArgs r) {
   __shared__ __align__(16) uint8_t rowbuf[kW][256];
@@ -695,7 +692,6 @@ __global__ void __launch_bounds__(kThreads) rot_tc_kernel(const __grid_constant_
   uint32_t sw = 0u;
   if (live && m < r.M) sw = rot_sign_bits(r.sign_bits, grp, lane);
   grid_dependency_wait();
-  for (int i = blockIdx.x * kThreads + tid; i < r.nclear; i += gridDim.x * kThreads) r.counters[i] = 0u;
   if (!live) return;  // warp-uniform
   uint8_t* row = rowbuf[warp];
   float sum = 0.f;
@@ -777,33 +773,34 @@ bool make_tc_plan(int B, int N, int K, int M, TcPlan& p) {
   const int xs_per_group = p.NT * 2048;
   const int red_bytes = kW * 3 * kTileRows * (8 * p.NT + 1) * 4;
   double best = -1.0;
-  for (int S = 1; S <= std::min(p.G, kSms); ++S) {
+  for (int S = 1; S <= std::min(p.G, kMaxCluster); ++S) {
     int L, d, nhi;
     if (!slice_lengths(p.G, S, B != 8, L, d, nhi)) continue;
     if (16 * B * L > 2048) continue;  // TMA box: at most 256 eight-byte elements per row
-    const int P = std::min(p.T, kSms / S);
+    const int P = std::min(p.T, kClustersAtOnce[S]);
     const int Tc = (p.T + P - 1) / P;
     const int U = Tc * L;
     const int uw = (U + kW - 1) / kW;
-    // busiest CTA: code bytes of its busiest warp times the warps, plus the
-    // slice partials it writes and reads back, plus the final sum's L2 round
-    // trips (one per kSliceBatch slices), each worth about 16 KB of streaming
+    // busiest CTA: code bytes of its busiest warp times the warps, plus (S > 1)
+    // the cluster's sum: two cluster barriers, each worth about 4 KB of
+    // streaming, and the slices' sums read from distributed shared memory
     const double cost = (double)uw * kW * kTileRows * 16 * B +
-                        (S > 1 ? (double)Tc * kTileRows * 8 * p.NT * 8 + 16384.0 * ((S + kSliceBatch - 1) / kSliceBatch)
-                               : 0.0);
+                        (S > 1 ? 8192.0 + (double)Tc * kTileRows * 8 * p.NT * 4 : 0.0);
     // shared memory
     const int tile_bytes = kTileRows * 16 * B * L;
     const int fixed = L * xs_per_group + ((L * 64 + 127) & ~127) + red_bytes + 64;
+    // per round tile: scale/zero pairs, the slice's tile sums (S > 1), the codes
+    auto per_tiles = [&](int k) {
+      return ((k * kTileRows * L * 4 + 127) & ~127) + (S > 1 ? ((k * kTileRows * 8 * p.NT * 4 + 127) & ~127) : 0);
+    };
     int RT, nbuf;
-    const int sz_all = (Tc * kTileRows * L * 4 + 127) & ~127;
-    if (fixed + sz_all + Tc * tile_bytes <= kSmemMax) {
+    if (fixed + per_tiles(Tc) + Tc * tile_bytes <= kSmemMax) {
       RT = Tc;
       nbuf = 1;
     } else {
       RT = 0;
       for (int k = Tc; k >= 1; --k) {
-        const int szk = (k * kTileRows * L * 4 + 127) & ~127;
-        if (fixed + szk + 2 * k * tile_bytes <= kSmemMax) {
+        if (fixed + per_tiles(k) + 2 * k * tile_bytes <= kSmemMax) {
           RT = k;
           break;
         }
@@ -829,21 +826,18 @@ bool make_tc_plan(int B, int N, int K, int M, TcPlan& p) {
   p.off_xsum = L * xs_per_group;
   p.off_sz = (p.off_xsum + L * 64 + 127) & ~127;
   p.off_red = (p.off_sz + p.RT * kTileRows * L * 4 + 127) & ~127;
-  p.off_codes = (p.off_red + red_bytes + 127) & ~127;
+  p.off_cp = (p.off_red + red_bytes + 127) & ~127;
+  const int cp_bytes = p.S > 1 ? p.RT * kTileRows * 8 * p.NT * 4 : 0;
+  p.off_codes = (p.off_cp + cp_bytes + 127) & ~127;
   p.off_bar = p.off_codes + p.nbuf * p.buf_bytes;
   p.smem_bytes = p.off_bar + 64;
   if (p.smem_bytes > kSmemMax) return false;
   // M >= 2: x rotated once per call (in-kernel rotation would repeat the
   // slice's M x L blocks in each of the P CTAs that share it)
   p.xrot = M >= 2 ? 1 : 0;
-  p.ws_part = ((size_t)p.T * 4 + 255) & ~(size_t)255;
-  const size_t part_end = p.ws_part + (p.S > 1 ? (size_t)p.T * p.S * kTileRows * 8 * p.NT * 4 : 0);
-  p.ws_xs = (part_end + 255) & ~(size_t)255;
-  p.ws_xsum = p.ws_xs + (size_t)p.G * p.NT * 2048;
-  if (p.xrot)
-    p.ws_total = p.ws_xsum + (size_t)p.G * 64;
-  else
-    p.ws_total = p.S > 1 ? part_end : 0;
+  p.ws_xs = 0;
+  p.ws_xsum = (size_t)p.G * p.NT * 2048;
+  p.ws_total = p.xrot ? p.ws_xsum + (size_t)p.G * 64 : 0;
   return true;
 }
 
@@ -863,11 +857,22 @@ qlin_status launch_tc_kernel(const TcArgs& a, cudaStream_t st) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = a.p.smem_bytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (a.p.S > 1) {  // the K slices of a row part (consecutive blocks) form one cluster
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = (unsigned)a.p.S;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (overlap_enabled()) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = overlap_enabled() ? 1 : 0;
+  cfg.numAttrs = na;
   return record_cuda(cudaLaunchKernelEx(&cfg, gemv_tc_kernel<B, NT>, a));
 }
 
@@ -939,8 +944,6 @@ qlin_status launch_gemv_tc(const PackedView& v, const __half* scales, const __ha
   a.x = x;
   a.y = y;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  a.counters = reinterpret_cast<uint32_t*>(ws);
-  a.part = a.p.S > 1 ? reinterpret_cast<float*>(ws + a.p.ws_part) : nullptr;
   a.xrot = a.p.xrot ? ws + a.p.ws_xs : nullptr;
   a.xsum_g = a.p.xrot ? reinterpret_cast<const float*>(ws + a.p.ws_xsum) : nullptr;
   a.N = v.N;
@@ -952,14 +955,9 @@ qlin_status launch_gemv_tc(const PackedView& v, const __half* scales, const __ha
     r.sign_bits = sign_bits;
     r.xrot = ws + a.p.ws_xs;
     r.xsum_g = reinterpret_cast<float*>(ws + a.p.ws_xsum);
-    r.counters = a.counters;
     r.M = M;
     r.K = v.K;
     r.G = a.p.G;
-    r.nclear = a.p.S > 1 ? a.p.T : 0;  // the rotation kernel zeroes the counters
-  } else if (a.p.S > 1) {
-    const cudaError_t e = cudaMemsetAsync(a.counters, 0, (size_t)a.p.T * 4, st);
-    if (e != cudaSuccess) return record_cuda(e);
   }
   switch (B) {
     case 3: return launch_tc_bits<3>(a, r, st);
