@@ -230,11 +230,6 @@ __device__ __forceinline__ uint64_t pk2(float lo, float hi) {
 __device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -268,9 +263,19 @@ __device__ __forceinline__ void copy_piece_any(int b, uint8_t* slot, const uint8
 }
 
 // ---- exact dequantisation of one 64-code piece (from the thread's ring slot) ----
-// q -> fp32 exactly through the bit pattern 2^23 + q (0x4B000000 | q) minus
-// 2^23; then t = q - z and p = s * t, each rounded to nearest in fp32 (the same
-// operations as dequant_exact, two lanes per instruction), then fp16.
+// Codes are cut out two at a time into the halves of a 32-bit word, each half
+// the 16-bit pattern m q with m a power of two (m q < 2048); one mixed-precision
+// fused multiply-add per code then gives fp32(q - z) 2^-9 and a packed multiply
+// by s 2^9 gives fp32(s t): the same two roundings as dequant_exact (see
+// fma_f16_f32 there), then fp16.  Which codes share a word depends on the
+// width:
+//   8 bits: bytes (4j + e, 4j + e + 1) of word j by one byte permute;
+//   4 bits: nibbles (8j + i, 8j + i + 4) of word j by one AND with 0x000F000F or
+//           0x00F000F0 (m = 1 or 16), half of them after a shift by 8;
+//   3 bits: codes (i, i + 8) from 27 bits starting at code i, AND 0x07000007
+//           (m = 1 and 256), for i = 16a + r, r < 8;
+//   6 bits: codes (i, i + 3), AND 0x00FC003F (m = 1 and 4), for i = 6a + r,
+//           r < 3, a < 10, and (60, 63); codes 61 and 62 by shifts.
 template <int B>
 __device__ __forceinline__ void dequant_piece(const uint8_t* piece, float s, float z, uint32_t (&out)[32]) {
   uint32_t w[2 * B + 1];
@@ -288,28 +293,56 @@ __device__ __forceinline__ void dequant_piece(const uint8_t* piece, float s, flo
     }
   }
   w[2 * B] = 0;
-  constexpr uint32_t kMask = (1u << B) - 1u;
-  const uint64_t c23 = pk2(8388608.0f, 8388608.0f), zz = pk2(z, z), ss = pk2(s, s);
+  // bits [bit, bit + 32) of the piece (zeros past its end)
+  auto bits_from = [&](int bit) -> uint32_t {
+    return (bit & 31) == 0 ? w[bit >> 5] : __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31);
+  };
+  const float zq = -z * 0x1p-9f;
+  float t[64];
+  if constexpr (B == 8) {
 #pragma unroll
-  for (int i = 0; i < 64; i += 2) {
-    uint32_t m[2];
+    for (int j = 0; j < 16; ++j) {
+      fma_f16x2_f32(__byte_perm(w[j], 0u, 0x4140u), kMul15, kMul15, zq, t[4 * j], t[4 * j + 1]);
+      fma_f16x2_f32(__byte_perm(w[j], 0u, 0x4342u), kMul15, kMul15, zq, t[4 * j + 2], t[4 * j + 3]);
+    }
+  } else if constexpr (B == 4) {
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int c = i + j;
-      if constexpr (B == 8) {
-        m[j] = __byte_perm(w[c >> 2], 0x4B000000u, 0x7540u | (uint32_t)(c & 3));
-      } else {
-        const int bit = B * c;
-        const uint32_t v = ((bit & 31) + B <= 32) ? (w[bit >> 5] >> (bit & 31))
-                                                  : __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31);
-        m[j] = (v & kMask) | 0x4B000000u;
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t v = w[j] >> 8;
+      fma_f16x2_f32(w[j] & 0x000F000Fu, kMul15, kMul15, zq, t[8 * j], t[8 * j + 4]);
+      fma_f16x2_f32(w[j] & 0x00F000F0u, kMul11, kMul11, zq, t[8 * j + 1], t[8 * j + 5]);
+      fma_f16x2_f32(v & 0x000F000Fu, kMul15, kMul15, zq, t[8 * j + 2], t[8 * j + 6]);
+      fma_f16x2_f32(v & 0x00F000F0u, kMul11, kMul11, zq, t[8 * j + 3], t[8 * j + 7]);
+    }
+  } else if constexpr (B == 3) {
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int i = 16 * a + r;
+        fma_f16x2_f32(bits_from(3 * i) & 0x07000007u, kMul15, kMul7, zq, t[i], t[i + 8]);
       }
     }
-    const uint64_t t = sub2(sub2(pk2(__uint_as_float(m[0]), __uint_as_float(m[1])), c23), zz);
+  } else {
+#pragma unroll
+    for (int a = 0; a < 10; ++a) {
+#pragma unroll
+      for (int r = 0; r < 3; ++r) {
+        const int i = 6 * a + r;
+        fma_f16x2_f32(bits_from(6 * i) & 0x00FC003Fu, kMul15, kMul13, zq, t[i], t[i + 3]);
+      }
+    }
+    const uint32_t v = w[11] >> 8;  // codes 60..63
+    fma_f16x2_f32(v & 0x00FC003Fu, kMul15, kMul13, zq, t[60], t[63]);
+    fma_f16x2_f32(((v >> 6) & 0x3Fu) | ((v << 4) & 0x003F0000u), kMul15, kMul15, zq, t[61], t[62]);
+  }
+  const uint64_t ss = pk2(s * 512.0f, s * 512.0f);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
     float p0, p1;
-    upk2(mul2(ss, t), p0, p1);
+    upk2(mul2(ss, pk2(t[2 * i], t[2 * i + 1])), p0, p1);
     __half2 h = __floats2half2_rn(p0, p1);
-    out[i >> 1] = *reinterpret_cast<uint32_t*>(&h);
+    out[i] = *reinterpret_cast<uint32_t*>(&h);
   }
 }
 

@@ -110,11 +110,37 @@ __device__ __forceinline__ uint32_t code_at(const uint32_t* row, int b, int k) {
   return q & ((1u << b) - 1u);
 }
 
-// fp16 weight: t = fp32(q) - z, p = s * t (each rounded to nearest in fp32, no
-// fused multiply-add), then one round-to-nearest-even to fp16.
+// fp32(a * b + c) with one rounding: a and b fp16 (bit patterns), c fp32.
+__device__ __forceinline__ float fma_f16_f32(uint16_t a, uint16_t b, float c) {
+  float d;
+  asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
+  return d;
+}
+
+// The two fp16 halves of x times b_lo and b_hi, plus c, each rounded once to fp32.
+__device__ __forceinline__ void fma_f16x2_f32(uint32_t x, uint16_t b_lo, uint16_t b_hi, float c, float& d_lo,
+                                              float& d_hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "fma.rn.f32.f16 %0, l, %3, %5;\n\tfma.rn.f32.f16 %1, h, %4, %5;\n\t}"
+      : "=f"(d_lo), "=f"(d_hi)
+      : "r"(x), "h"(b_lo), "h"(b_hi), "f"(c));
+}
+
+// Subtraction of the zero point rounded exactly as fp32(q) - z, scaled by 2^-9:
+//   fma_f16_f32(m q, 2^15 / m, -z 2^-9) = fp32(q - z) * 2^-9.
+// The 16-bit pattern m q (< 2048) is the fp16 number m q 2^-24 (subnormal, or
+// exponent field 1, where the value still grows by 2^-24 per step); times the
+// fp16 multiplier 2^15 / m it is q 2^-9 exactly, and the fused add rounds
+// q 2^-9 - z 2^-9 once.  Scaling by a power of two commutes with rounding while
+// the result stays normal, which it does: |q - z| >= 2^-24 unless it is 0.
+constexpr uint16_t kMul15 = 0x7800, kMul13 = 0x7000, kMul11 = 0x6800, kMul7 = 0x5800;  // 2^15, 2^13, 2^11, 2^7
+
+// fp16 weight: t = fp32(q) - z, p = s * t (each rounded to nearest in fp32),
+// then one round-to-nearest-even to fp16.  t comes from the form above and p from
+// (s 2^9) * (t 2^-9): both scalings are exact, so p is the same fp32 number.
 __device__ __forceinline__ __half dequant_exact(uint32_t q, float s, float z) {
-  const float t = __fsub_rn(__uint2float_rn(q), z);
-  const float p = __fmul_rn(s, t);
+  const float t9 = fma_f16_f32((uint16_t)q, kMul15, -z * 0x1p-9f);
+  const float p = __fmul_rn(s * 512.0f, t9);
   return __float2half_rn(p);
 }
 

@@ -8,6 +8,8 @@ int4, down-proj int3 at M = 1/4/16, the 36-layer int6 stack with the int8
 lm_head, the mixed int6/int8 prefill GEMM at M = 256/1024/2048) plus ragged
 and degenerate shapes.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -94,6 +96,51 @@ def test_dequant_bit_exact_adversarial_scales():
     got = Q.qlin_dequant(d, packed, torch.from_numpy(s).to(DEV), torch.from_numpy(z).to(DEV)).cpu().numpy()
     ref = O.dequant16(codes, s, z)
     assert got.view(np.uint16).tobytes() == ref.view(np.uint16).tobytes()
+
+
+def _wide_zero_points(rng, shape):
+    """fp16 zero points of every magnitude, subnormals included, either sign."""
+    z = np.exp(rng.uniform(-17.5, 6.0, shape)) * rng.choice([-1.0, 1.0], shape)
+    return z.astype(np.float16)
+
+
+@pytest.mark.parametrize("bits", [3, 4, 6, 8])
+def test_dequant_bit_exact_tiny_zero_points(bits):
+    """Zero points down to the fp16 subnormals: fp32(q) - z is then often not
+    exact, so the two fp32 roundings (subtract, multiply) both show."""
+    rng = np.random.default_rng(11 + bits)
+    N, K = 96, 512
+    codes = rng.integers(0, 1 << bits, size=(N, K), dtype=np.uint8)
+    s = (np.exp(rng.uniform(-14, 3, (N, K // 128))) * rng.choice([-1.0, 1.0], (N, K // 128))).astype(np.float16)
+    z = _wide_zero_points(rng, (N, K // 128))
+    zk = np.repeat(z.astype(np.float64), 128, axis=1)
+    inexact = (codes.astype(np.float32) - zk.astype(np.float32)).astype(np.float64) != codes - zk
+    assert inexact.mean() > 0.05
+    d = Q.Desc(N, K, bits)
+    packed = Q.qlin_pack(d, torch.from_numpy(codes).to(DEV))
+    got = Q.qlin_dequant(d, packed, torch.from_numpy(s).to(DEV), torch.from_numpy(z).to(DEV)).cpu().numpy()
+    ref = O.dequant16(codes, s, z)
+    assert got.view(np.uint16).tobytes() == ref.view(np.uint16).tobytes()
+
+
+@pytest.mark.parametrize("bits", [3, 4, 6, 8])
+def test_gemm_wide_zero_points(bits):
+    """The GEMM dequantises in tensor memory with its own code extraction:
+    arbitrary zero points (tiny, subnormal, negative, large) and scales of
+    either sign, against the oracle."""
+    rng = np.random.default_rng(21 + bits)
+    N, K, M = 320, 1280, 96
+    w = _rand_weight(N, K, bits, seed=5 + bits)
+    G = K // 128
+    s = (np.exp(rng.uniform(-12, -6, (N, G))) * rng.choice([-1.0, 1.0], (N, G))).astype(np.float16)
+    z = _wide_zero_points(rng, (N, G))
+    w = dataclasses.replace(w, scales=torch.from_numpy(s).to(DEV), zeros=torch.from_numpy(z).to(DEV))
+    a = W.draw_activation(M, K, seed=bits).to(DEV)
+    d, packed = packed_on_device(w)
+    y = Q.qlin_gemm(d, packed, w.scales, w.zeros, a.sign_bits, a.x)
+    torch.cuda.synchronize()
+    assert_close(y, oracle_rows(w, a), f"gemm wide zeros b{bits}")
+    assert_dot_bound(y, w, a, what=f"gemm wide zeros b{bits}")
 
 
 # ------------------------------------------------------------------- rht ------
