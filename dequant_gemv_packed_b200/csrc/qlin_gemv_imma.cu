@@ -33,9 +33,10 @@
 //   * 16 consumer warps: rotate x (one block of 128 per warp at a time, on the
 //     tensor cores: qlin_rot16.cuh), write each group's digit planes and
 //     (xs, xs X) to shared memory, then take (16-row tile, group pair) items
-//     from a shared counter; each item's two output partial sums go to a
-//     shared [pair][row] array, which is summed over pairs in a fixed order
-//     at the end (deterministic results whatever warp took which item).
+//     in tile-major order, one contiguous range per warp; over its run of
+//     items of one tile a lane keeps its rows' partial sums in registers and
+//     writes them once to a shared [warp][row] array, which is summed over
+//     the warps in a fixed order at the end (deterministic results).
 // With qlin_set_overlap(1) the kernel is a programmatic dependent, like the
 // other M = 1 kernel: the weight stream starts before the previous kernel
 // ends; x is read, and y written, after it.
@@ -72,7 +73,7 @@ struct ImmaPlan {
   int tile_bytes;      // stride of the tiles in shared memory (a multiple of 128)
   int sz_halves;       // halves per array (scales, zeros) in shared memory
   int inflight;        // tiles whose copies the producer has in flight at once
-  int off_sz, off_xb, off_xc, off_part, off_bar;
+  int off_sz, off_xb, off_xc, off_part, off_x, off_bar;
   int smem_bytes;
 };
 
@@ -112,19 +113,6 @@ __device__ __forceinline__ float ldsh2f(uint32_t addr) {
   uint16_t h;
   asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h) : "r"(addr));
   return __half2float(__ushort_as_half(h));
-}
-
-// The partial sums of this lane's rows (tile rows la and la + 4) for its group
-// (lanes t = 0, 1; `valid` false: no group), added over the pair's two groups
-// and stored by lane t = 0 at part[idx] and part[idx + 4].
-__device__ __forceinline__ void store_pair(float* part, int idx, float pa, float pb, bool valid, int t) {
-  if (!valid) pa = pb = 0.f;
-  pa += __shfl_xor_sync(0xffffffffu, pa, 1);
-  pb += __shfl_xor_sync(0xffffffffu, pb, 1);
-  if (t == 0) {
-    part[idx] = pa;
-    part[idx + 4] = pb;
-  }
 }
 
 // Where code c (0..127) of a group sits in a digit plane.  Lane t's 32 bytes
@@ -192,20 +180,21 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
   uint8_t* xb = smem + p.off_xb;            // [G][288]: digit planes (high at 0, low at 144), then 32 zero bytes
   uint8_t* zero32 = xb + (size_t)G * kGroupXB;
   float2* xc = reinterpret_cast<float2*>(smem + p.off_xc);
-  float* part = reinterpret_cast<float*>(smem + p.off_part);  // [GP][Rp]
+  float* part = reinterpret_cast<float*>(smem + p.off_part);  // [kNW][Rp]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   uint64_t* sz_full = full + kMaxTiles;
   uint64_t* x_issued = sz_full + 1;
-  int* counter = reinterpret_cast<int*>(x_issued + 1);
+  uint64_t* x_full = x_issued + 1;
+  const __half* xs = reinterpret_cast<const __half*>(smem + p.off_x);  // x, copied in once
 
   if (tid == kNW * 32) {
     for (int r = 0; r < T; ++r) mbar_init(&full[r], 1);
     mbar_init(sz_full, 1);
-    mbar_init(x_issued, kNW);
+    mbar_init(x_issued, 1);
+    mbar_init(x_full, 1);
     mbar_fence_init();
   }
   if (tid < 8) reinterpret_cast<uint32_t*>(zero32)[tid] = 0u;
-  if (tid == 0) *counter = 0;
   __syncthreads();
   if (tid == 0) grid_launch_dependents();
 
@@ -248,9 +237,10 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
   }
 
   // ------------------------------------------------------------- prologue --
-  // Blocks g = warp, warp + 16, ...: all of the warp's x loads are issued
-  // before any is used (one memory latency).  The sign bits (weights side) are
-  // read before the dependency wait, x after it.
+  // x arrives in one bulk copy, issued by thread 0 right after the dependency
+  // wait (one request per CTA for the vector every CTA reads, instead of one
+  // per warp and block); the sign bits (weights side) are read before it.
+  // Blocks g = warp, warp + 16, ... are then rotated from shared memory.
   {
     uint32_t h[4];
     h16_fragment(lane, h);
@@ -262,17 +252,21 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
         const int blk = min(blk0 + j * kNW, G - 1);
         sw[j] = rot_sign_bits(a.sign_bits, blk, lane);
       }
-      if (blk0 == warp) grid_dependency_wait();
+      if (blk0 == warp) {
+        if (tid == 0) {
+          grid_dependency_wait();
+          mbar_arrive_expect_tx(x_full, 2u * (uint32_t)a.K);
+          bulk_g2s(const_cast<__half*>(xs), a.x, 2u * (uint32_t)a.K, x_full);
+          mbar_arrive(x_issued);
+        }
+        if (!mbar_wait(x_full, 0, &g_imma_error)) imma_fail(0x40u);
+      }
 #pragma unroll
       for (int j = 0; j < kXBatch; ++j) {
         const int blk = min(blk0 + j * kNW, G - 1);
-        const __half* xp = a.x + (size_t)blk * kHadamard + xo;
+        const __half* xp = xs + (size_t)blk * kHadamard + xo;
         xb0[j] = *reinterpret_cast<const uint32_t*>(xp);
         xb1[j] = *reinterpret_cast<const uint32_t*>(xp + 8);
-      }
-      if (blk0 == warp) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(x_issued);
       }
 #pragma unroll
       for (int j = 0; j < kXBatch; ++j) {
@@ -281,19 +275,18 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
         prepare_group<B>(xb0[j], xb1[j], sw[j], h, lane, xb + (size_t)blk * kGroupXB, xc + blk);
       }
     }
-    if (warp >= G) {  // a warp with no block has nothing to load
-      grid_dependency_wait();
-      if (lane == 0) mbar_arrive(x_issued);
-    }
   }
   named_barrier(1, kNW * 32);  // digit planes and (xs, xs X) of every group written
   if (!mbar_wait(sz_full, 0, &g_imma_error)) imma_fail(0x20u);
 
   // ------------------------------------------------------------ main loop --
-  // Items (group pair pp, tile r) in pair-major order, item = pp T + r; warp w
-  // takes the contiguous range [w I / 16, (w + 1) I / 16), so that it loads a
-  // pair's B fragments and x scalars once for all of its tiles of that pair.
-  // Shared memory is addressed with 32-bit offsets computed once per lane.
+  // Items (16-row tile r, group pair pp) in tile-major order, item = r GP + pp;
+  // warp w takes the contiguous range [w I / 16, (w + 1) I / 16).  Over a run
+  // of items of one tile each lane keeps its two rows' partial sums in
+  // registers (lanes t = 0, 1: groups 2 pp + t), so an item is one chain of
+  // loads, MMAs and two multiply-adds; at the end of the run the two lanes'
+  // sums are added and written once, to part[w][row].  A tile's barrier is
+  // tested once per run.  Shared memory is addressed with 32-bit offsets.
   const int I = T * GP;
   const int i0 = (int)(((long long)warp * I) / kNW), i1 = (int)(((long long)(warp + 1) * I) / kNW);
   const int slot = gl >> 1;  // this lane's B column: (slot, digit) = (gl / 2, gl % 2)
@@ -306,47 +299,47 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
   const uint32_t row4 = 4u * (uint32_t)p.row_bytes;
   const uint32_t s_u = smem_addr(s_raw), z_u = smem_addr(z_raw);
   const int sz_off = (int)(((size_t)n0 * G) & 7);  // the CTA's first scale in its aligned copy
-  int pp = i0 / T, r = i0 - pp * T;
-  int cur_pp = -1;
-  unsigned long long waited = 0ull;
-  uint4 b0A = {}, b0B = {}, b1A = {}, b1B = {};
-  float2 xv = make_float2(0.f, 0.f);
-  bool has1 = false;
-  int gq = 0;
+  int r = i0 / GP, pp = i0 - r * GP;
+  bool at_run_start = true;
+  uint32_t ra_u = 0, rb_u = 0;
+  int ra = 0, rb = 0;
+  float acc_a = 0.f, acc_b = 0.f;
   for (int it = i0; it < i1; ++it) {
-    if (pp != cur_pp) {  // warp-uniform: a new pair
-      cur_pp = pp;
-      const int g0 = 2 * pp;
-      has1 = g0 + 1 < G;
-      const uint32_t b0 = slot == 0 ? xb_lane + (uint32_t)(g0 * kGroupXB) : zero_u;
-      const uint32_t b1 = (slot == 1 && has1) ? xb_lane + (uint32_t)((g0 + 1) * kGroupXB) : zero_u;
-      b0A = ldsu128(b0);
-      b0B = ldsu128(b0 + 16);
-      b1A = ldsu128(b1);
-      b1B = ldsu128(b1 + 16);
-      gq = (t == 1 && has1) ? g0 + 1 : g0;  // lanes t = 0, 1: group g0 + t
-      xv = xc[gq];
-    }
-    if (!((waited >> r) & 1ull)) {  // warp-uniform
+    if (at_run_start) {  // warp-uniform: this warp's first item of tile r
+      at_run_start = false;
       if (!mbar_wait_poll(&full[r], 0, &g_imma_error)) imma_fail(0x10u);
-      waited |= 1ull << r;
-    }
-    // this lane's two rows (in the last tile, rows past the share read the last row)
-    const uint32_t tile_u = code0 + (uint32_t)r * (uint32_t)p.tile_bytes;
-    uint32_t ra_u = tile_u + lane_row, rb_u = ra_u + row4;
-    int ra = 16 * r + la, rb = ra + 4;
-    if (rb > R - 1) {
-      const int lr = R - 1 - 16 * r;
-      const uint32_t last = tile_u + (uint32_t)((lr >> 3) * p.chunk_b + (lr & 7) * p.row_bytes);
-      if (ra > R - 1) {
-        ra = R - 1;
-        ra_u = last;
+      // this lane's two rows (in the last tile, rows past the share read the last row)
+      const uint32_t tile_u = code0 + (uint32_t)r * (uint32_t)p.tile_bytes;
+      ra_u = tile_u + lane_row;
+      rb_u = ra_u + row4;
+      ra = 16 * r + la;
+      rb = ra + 4;
+      if (rb > R - 1) {
+        const int lr = R - 1 - 16 * r;
+        const uint32_t last = tile_u + (uint32_t)((lr >> 3) * p.chunk_b + (lr & 7) * p.row_bytes);
+        if (ra > R - 1) {
+          ra = R - 1;
+          ra_u = last;
+        }
+        rb = R - 1;
+        rb_u = last;
       }
-      rb = R - 1;
-      rb_u = last;
     }
-    const uint32_t g0b = (uint32_t)(2 * pp * kGroupBytes);
+    const int g0 = 2 * pp;
+    const bool has1 = g0 + 1 < G;
+    const int gq = (t == 1 && has1) ? g0 + 1 : g0;  // lanes t = 0, 1: group g0 + t
+    const uint32_t b0 = slot == 0 ? xb_lane + (uint32_t)(g0 * kGroupXB) : zero_u;
+    const uint32_t b1 = (slot == 1 && has1) ? xb_lane + (uint32_t)((g0 + 1) * kGroupXB) : zero_u;
+    const uint4 b0A = ldsu128(b0), b0B = ldsu128(b0 + 16);
+    const uint4 b1A = ldsu128(b1), b1B = ldsu128(b1 + 16);
+    const float sa = ldsh2f(s_u + 2u * (uint32_t)(sz_off + ra * G + gq));
+    const float za = ldsh2f(z_u + 2u * (uint32_t)(sz_off + ra * G + gq));
+    const float sb = ldsh2f(s_u + 2u * (uint32_t)(sz_off + rb * G + gq));
+    const float zb = ldsh2f(z_u + 2u * (uint32_t)(sz_off + rb * G + gq));
+    const float2 xv = xc[gq];
+    const uint32_t g0b = (uint32_t)(g0 * kGroupBytes);
     int dl[4] = {0, 0, 0, 0}, dh[4] = {0, 0, 0, 0};
+    int Sa, Sb;
     if constexpr (B == 4) {
       const uint4 wa0 = ldsu128(ra_u + g0b), wb0 = ldsu128(rb_u + g0b);
       uint4 wa1 = {}, wb1 = {};
@@ -354,10 +347,6 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
         wa1 = ldsu128(ra_u + g0b + kGroupBytes);
         wb1 = ldsu128(rb_u + g0b + kGroupBytes);
       }
-      const float sa = ldsh2f(s_u + 2u * (uint32_t)(sz_off + ra * G + gq));
-      const float za = ldsh2f(z_u + 2u * (uint32_t)(sz_off + ra * G + gq));
-      const float sb = ldsh2f(s_u + 2u * (uint32_t)(sz_off + rb * G + gq));
-      const float zb = ldsh2f(z_u + 2u * (uint32_t)(sz_off + rb * G + gq));
       constexpr uint32_t kLo = 0x0F0F0F0Fu, kHi = 0xF0F0F0F0u;
       mma_u8s8(dl, wa0.x & kLo, wb0.x & kLo, wa0.y & kLo, wb0.y & kLo, b0A.x, b0A.y);
       mma_u8s8(dh, wa0.x & kHi, wb0.x & kHi, wa0.y & kHi, wb0.y & kHi, b0B.x, b0B.y);
@@ -370,15 +359,9 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
         mma_u8s8(dh, wa1.z & kHi, wb1.z & kHi, wa1.w & kHi, wb1.w & kHi, b1B.z, b1B.w);
       }
       // lane (gl, t < 2): rows ra, rb of group g0 + t; columns 2t (high digit), 2t + 1 (low digit)
-      const int Sa = ((dl[0] + (dh[0] >> 4)) << 8) + (dl[1] + (dh[1] >> 4));
-      const int Sb = ((dl[2] + (dh[2] >> 4)) << 8) + (dl[3] + (dh[3] >> 4));
-      store_pair(part, pp * Rp + 16 * r + la, sa * fmaf(-za, xv.y, xv.x * (float)Sa),
-                 sb * fmaf(-zb, xv.y, xv.x * (float)Sb), t == 0 || (t == 1 && has1), t);
+      Sa = ((dl[0] + (dh[0] >> 4)) << 8) + (dl[1] + (dh[1] >> 4));
+      Sb = ((dl[2] + (dh[2] >> 4)) << 8) + (dl[3] + (dh[3] >> 4));
     } else {
-      const float sa = ldsh2f(s_u + 2u * (uint32_t)(sz_off + ra * G + gq));
-      const float za = ldsh2f(z_u + 2u * (uint32_t)(sz_off + ra * G + gq));
-      const float sb = ldsh2f(s_u + 2u * (uint32_t)(sz_off + rb * G + gq));
-      const float zb = ldsh2f(z_u + 2u * (uint32_t)(sz_off + rb * G + gq));
       {
         const uint4 wa0 = ldsu128(ra_u + g0b), wa1 = ldsu128(ra_u + g0b + 16);
         const uint4 wb0 = ldsu128(rb_u + g0b), wb1 = ldsu128(rb_u + g0b + 16);
@@ -396,29 +379,42 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_imma_kernel(const __grid_con
         mma_u8s8(dh, wa3.z, wb3.z, wa3.w, wb3.w, b1B.z, b1B.w);
       }
       // two accumulators for latency only: both hold plain sums
-      const int Sa = ((dl[0] + dh[0]) << 8) + (dl[1] + dh[1]);
-      const int Sb = ((dl[2] + dh[2]) << 8) + (dl[3] + dh[3]);
-      store_pair(part, pp * Rp + 16 * r + la, sa * fmaf(-za, xv.y, xv.x * (float)Sa),
-                 sb * fmaf(-zb, xv.y, xv.x * (float)Sb), t == 0 || (t == 1 && has1), t);
+      Sa = ((dl[0] + dh[0]) << 8) + (dl[1] + dh[1]);
+      Sb = ((dl[2] + dh[2]) << 8) + (dl[3] + dh[3]);
     }
-    if (++r == T) {
-      r = 0;
-      ++pp;
+    if (t == 0 || (t == 1 && has1)) {
+      acc_a += sa * fmaf(-za, xv.y, xv.x * (float)Sa);
+      acc_b += sb * fmaf(-zb, xv.y, xv.x * (float)Sb);
+    }
+    if (++pp == GP || it + 1 == i1) {  // warp-uniform: the end of this warp's run of tile r
+      acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 1);
+      acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 1);
+      if (t == 0) {
+        part[warp * Rp + 16 * r + la] = acc_a;
+        part[warp * Rp + 16 * r + la + 4] = acc_b;
+      }
+      acc_a = acc_b = 0.f;
+      if (pp == GP) {
+        pp = 0;
+        ++r;
+        at_run_start = true;
+      }
     }
   }
   named_barrier(1, kNW * 32);
 
   // ---------------------------------------------------------- row sums ----
-  // Four threads per row, each a fixed stride of the pairs, then two shuffles:
-  // a fixed summation order.
-  for (int base = 0; base < R; base += kNW * 8) {
-    const int row = base + (tid >> 2), sub = tid & 3;
+  // Row n0 + row of tile r: the sum of part[w][row] over the warps w whose
+  // item ranges meet the tile's items [r GP, (r + 1) GP), in warp order.
+  // Item x lies in the range of warp (16 x + 15) / I.
+  for (int row = tid; row < R; row += kNW * 32) {
+    const int rt = row >> 4;
+    const int w_lo = (kNW * rt * GP + kNW - 1) / I;
+    const int w_hi = (kNW * ((rt + 1) * GP - 1) + kNW - 1) / I;
     float acc = 0.f;
-    if (row < R)
-      for (int q = sub; q < GP; q += 4) acc += part[q * Rp + row];
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (sub == 0 && row < R) a.y[n0 + row] = __float2half_rn(acc);
+    for (int w = w_lo; w <= w_hi; ++w)
+      if ((long long)w * I / kNW < (long long)(w + 1) * I / kNW) acc += part[w * Rp + row];
+    a.y[n0 + row] = __float2half_rn(acc);
   }
 }
 
@@ -449,7 +445,8 @@ bool make_imma_plan(int b, int N, int K, ImmaPlan& p) {
   p.off_xb = (p.off_sz + 4 * p.sz_halves + 127) & ~127;
   p.off_xc = (p.off_xb + p.G * kGroupXB + 32 + 15) & ~15;
   p.off_part = (p.off_xc + p.G * 8 + 127) & ~127;
-  p.off_bar = (p.off_part + p.GP * 16 * p.T * 4 + 127) & ~127;
+  p.off_x = (p.off_part + kNW * 16 * p.T * 4 + 127) & ~127;
+  p.off_bar = (p.off_x + 2 * K + 127) & ~127;
   p.inflight = kInflightTiles;
   const int end = p.off_bar + (kMaxTiles + 2) * 8 + 16;
   p.smem_bytes = std::max(end, kMinSmem);
