@@ -404,6 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
+      grid_dependency_wait();  // the rotated activations are the rotation kernel's output
       int g = 0, t, g0, g1;
       Segments sg;
       sg.init(a);
@@ -448,6 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     // --------------------------------------------------------- epilogue --
     const int q = warp & 3;  // TMEM lanes 32q..32q+31 = weight rows of the tile
     const int row = 32 * q + lane;
+    grid_dependency_wait();  // the completion flags are cleared by the rotation kernel
     const long long T = (long long)tiles * (a.v.K / kGroup);
     const int G = a.v.K / kGroup, P = gridDim.x, c = blockIdx.x;
     // The accumulator is handed back to the MMA as soon as this warp has
@@ -734,8 +736,20 @@ qlin_status launch_gemm_rotated(const PackedView& v, const __half* scales, const
   const long long tiles = (long long)a.m_tiles * a.n_tiles;
   const long long work = a.stream_k ? tiles * (v.K / kGroup) : tiles;
   const int grid = (int)std::min<long long>(work, kSms);
-  gemm_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(map, ymap, a);
-  return record_cuda(cudaGetLastError());
+  // A programmatic dependent of the rotation kernel: set-up, tensor memory and
+  // the first stages' dequantisation (weights only) overlap the rotation; the
+  // TMA producer and the epilogue wait for it before they read its output.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return record_cuda(cudaLaunchKernelEx(&cfg, gemm_tc_kernel, map, ymap, a));
 }
 
 qlin_status launch_gemm(const PackedView& v, const __half* scales, const __half* zeros,

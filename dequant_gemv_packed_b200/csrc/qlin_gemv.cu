@@ -186,14 +186,14 @@ __device__ __forceinline__ float dot_unit(const uint32_t (&w)[12], const uint32_
     const uint32_t x01 = x[4 * p], x23 = x[4 * p + 1], x45 = x[4 * p + 2], x67 = x[4 * p + 3];
     float& A1 = (p & 1) ? a1b : a1a;
     float& A4 = (p & 1) ? a4b : a4a;
-    A1 = fma_f16f32(lo16(T0), lo16(x01), A1);
-    A4 = fma_f16f32(hi16(T0), hi16(x23), A4);
-    A1 = fma_f16f32(lo16(T1), hi16(x01), A1);
-    A4 = fma_f16f32(hi16(T1), lo16(x45), A4);
-    A1 = fma_f16f32(lo16(T2), lo16(x23), A1);
-    A4 = fma_f16f32(hi16(T2), hi16(x45), A4);
-    A1 = fma_f16f32(lo16(T3), lo16(x67), A1);
-    A4 = fma_f16f32(hi16(T3), hi16(x67), A4);
+    A1 = fma_f16_f32(lo16(T0), lo16(x01), A1);
+    A4 = fma_f16_f32(hi16(T0), hi16(x23), A4);
+    A1 = fma_f16_f32(lo16(T1), hi16(x01), A1);
+    A4 = fma_f16_f32(hi16(T1), lo16(x45), A4);
+    A1 = fma_f16_f32(lo16(T2), lo16(x23), A1);
+    A4 = fma_f16_f32(hi16(T2), hi16(x45), A4);
+    A1 = fma_f16_f32(lo16(T3), lo16(x67), A1);
+    A4 = fma_f16_f32(hi16(T3), hi16(x67), A4);
   }
   return (a1a + a1b) + 0.25f * (a4a + a4b);
 }
@@ -217,22 +217,22 @@ __device__ __forceinline__ float dot_unit(const uint32_t (&w)[6], const uint32_t
     const uint32_t T6 = (R & 0x00070007u) | kMagic;   // (q3, q11)
     const uint32_t T7 = (R & 0x00380038u) | kMagic;   // (8 q4, 8 q12)
     const uint32_t* xp = x + 8 * p;  // xp[i] = (x_{2i}, x_{2i+1}) of this piece
-    a2 = fma_f16f32(lo16(T0), lo16(xp[0]), a2);
-    a1 = fma_f16f32(hi16(T0), hi16(xp[2]), a1);
-    a16 = fma_f16f32(lo16(T1), hi16(xp[0]), a16);
-    a8 = fma_f16f32(hi16(T1), lo16(xp[3]), a8);
-    a128 = fma_f16f32(lo16(T2), lo16(xp[1]), a128);
-    a64 = fma_f16f32(hi16(T2), hi16(xp[3]), a64);
-    a2 = fma_f16f32(lo16(T3), lo16(xp[4]), a2);
-    a1 = fma_f16f32(hi16(T3), hi16(xp[6]), a1);
-    a16 = fma_f16f32(lo16(T4), hi16(xp[4]), a16);
-    a8 = fma_f16f32(hi16(T4), lo16(xp[7]), a8);
-    a128 = fma_f16f32(lo16(T5), lo16(xp[5]), a128);
-    a64 = fma_f16f32(hi16(T5), hi16(xp[7]), a64);
-    a1 = fma_f16f32(lo16(T6), hi16(xp[1]), a1);
-    a1 = fma_f16f32(hi16(T6), hi16(xp[5]), a1);
-    a8 = fma_f16f32(lo16(T7), lo16(xp[2]), a8);
-    a8 = fma_f16f32(hi16(T7), lo16(xp[6]), a8);
+    a2 = fma_f16_f32(lo16(T0), lo16(xp[0]), a2);
+    a1 = fma_f16_f32(hi16(T0), hi16(xp[2]), a1);
+    a16 = fma_f16_f32(lo16(T1), hi16(xp[0]), a16);
+    a8 = fma_f16_f32(hi16(T1), lo16(xp[3]), a8);
+    a128 = fma_f16_f32(lo16(T2), lo16(xp[1]), a128);
+    a64 = fma_f16_f32(hi16(T2), hi16(xp[3]), a64);
+    a2 = fma_f16_f32(lo16(T3), lo16(xp[4]), a2);
+    a1 = fma_f16_f32(hi16(T3), hi16(xp[6]), a1);
+    a16 = fma_f16_f32(lo16(T4), hi16(xp[4]), a16);
+    a8 = fma_f16_f32(hi16(T4), lo16(xp[7]), a8);
+    a128 = fma_f16_f32(lo16(T5), lo16(xp[5]), a128);
+    a64 = fma_f16_f32(hi16(T5), hi16(xp[7]), a64);
+    a1 = fma_f16_f32(lo16(T6), hi16(xp[1]), a1);
+    a1 = fma_f16_f32(hi16(T6), hi16(xp[5]), a1);
+    a8 = fma_f16_f32(lo16(T7), lo16(xp[2]), a8);
+    a8 = fma_f16_f32(hi16(T7), lo16(xp[6]), a8);
   }
   return a1 + 0.5f * a2 + 0.125f * a8 + 0.0625f * a16 + 0.015625f * a64 + 0.0078125f * a128;
 }

@@ -7,6 +7,7 @@
 // inference on CUDA", paragraph "Random Hadamard transform").  One warp per
 // (row, block); the transform is tiny next to the matmul it feeds.
 #include "qlin_internal.cuh"
+#include "qlin_sm100.cuh"
 
 namespace qlin {
 
@@ -14,6 +15,10 @@ __global__ void rht_kernel(const __half* __restrict__ x, __half* __restrict__ xr
                            const uint32_t* __restrict__ sign_bits, int M, int K, uint32_t* clear, int nclear,
                            float* xsum) {
   const int lane = threadIdx.x & 31;
+  // A kernel launched after this one as a programmatic dependent (the GEMM)
+  // may start now: it reads what this kernel writes only after its own
+  // dependency wait.
+  if (threadIdx.x == 0) grid_launch_dependents();
   // Words the kernel that follows expects to find zero (its completion flags).
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < nclear; i += blockDim.x) clear[i] = 0u;

@@ -122,13 +122,6 @@ __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// d = a * b + c with fp16 a, b and fp32 c, d (one rounding, in fp32).
-__device__ __forceinline__ float fma_f16f32(uint16_t a, uint16_t b, float c) {
-  float d;
-  asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
-  return d;
-}
-
 __device__ __forceinline__ uint16_t lo16(uint32_t v) {
   uint16_t lo;
   asm("{\n\t.reg .b16 t;\n\tmov.b32 {%0, t}, %1;\n\t}" : "=h"(lo) : "r"(v));
