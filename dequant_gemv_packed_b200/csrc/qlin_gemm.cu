@@ -510,16 +510,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           // acquire in every lane before its loads of the partial
           asm volatile("{\n\t.reg .b32 f;\n\tld.acquire.gpu.global.u32 f, [%0];\n\t}" ::"l"(a.flags + cc) : "memory");
         }
-        for (int c0 = 0; c0 < a.BN; c0 += 32) {
+        // The later contributors' partials, one (chunk, contributor) after the
+        // other in that order, each loaded while the one before is added.
+        const int ncon = c_last - c, nk = ncon * ((a.BN + 31) / 32);
+        float nxt[32];
+        auto load_part = [&](int k) {
+          const float* src =
+              a.partials + (size_t)(c + 1 + k % ncon) * a.part_cols * kBMw + (size_t)(32 * (k / ncon)) * kBMw + row;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) nxt[j] = __ldcg(src + (size_t)j * kBMw);
+        };
+        if (nk > 0) load_part(0);
+        for (int c0 = 0, k = 0; c0 < a.BN; c0 += 32) {
           uint32_t r[32];
           tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCol + c0), r);
           float acc[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(r[j]);
-          for (int cc = c + 1; cc <= c_last; ++cc) {
-            const float* src = a.partials + (size_t)cc * a.part_cols * kBMw + (size_t)c0 * kBMw + row;
+          for (int cc = 0; cc < ncon; ++cc, ++k) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) acc[j] += __ldcg(src + (size_t)j * kBMw);
+            for (int j = 0; j < 32; ++j) acc[j] += nxt[j];
+            if (k + 1 < nk) load_part(k + 1);
           }
           if (a.tma_store) {
             // the whole tile is staged (fp16, [m][n]) and stored by one thread
