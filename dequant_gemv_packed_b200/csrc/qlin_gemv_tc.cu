@@ -106,9 +106,31 @@ struct RotArgs {
   uint8_t* xrot;       // [G][NT][8][256 B]
   float* xsum_g;       // [G][16]
   int M, K, G;
+  // the layer's weight arrays (codes, scales, zeros) and their sizes in bytes,
+  // prefetched into L2 for the GEMV that follows
+  const void* pf[3];
+  size_t pf_bytes[3];
 };
 
 __device__ __forceinline__ void tc_fail(unsigned code) { atomicOr(&g_tc_error, code); }
+
+// Hint: bring [p, p + bytes) into L2 (p and bytes multiples of 16).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Lane `lane` of one warp per CTA prefetches its share of the CTA's slice
+// [n b / nb, n (b + 1) / nb) of an array of n bytes (16-byte aligned), in
+// pieces of at most 32 KB, ending on 16-byte boundaries.
+__device__ __forceinline__ void prefetch_l2_share(const void* base, size_t n, int b, int nb, int lane) {
+  if (base == nullptr || n < 16) return;
+  const size_t lo = (n * (size_t)b / (size_t)nb) & ~(size_t)15, hi = (n * (size_t)(b + 1) / (size_t)nb) & ~(size_t)15;
+  constexpr size_t kPiece = 32768;
+  for (size_t o = lo + (size_t)lane * kPiece; o < hi; o += 32 * kPiece) {
+    const size_t len = hi - o < kPiece ? hi - o : kPiece;
+    prefetch_l2(static_cast<const uint8_t*>(base) + o, (uint32_t)len);
+  }
+}
 
 // Barrier of every thread of every CTA of the cluster; shared-memory writes
 // before it are visible to the cluster's loads after it.
@@ -686,6 +708,12 @@ __global__ void __launch_bounds__(kThreads) rot_tc_kernel(const __grid_constant_
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   if (tid == 0) grid_launch_dependents();
+  // Launched as a programmatic dependent, this kernel starts while the kernel
+  // before it still runs, and waits for it below; before that wait, warp 0
+  // brings this CTA's share of the layer's weights into L2, so that the
+  // GEMV's tensor loads after this kernel find them there.
+  if (warp == 0)
+    for (int i = 0; i < 3; ++i) prefetch_l2_share(r.pf[i], r.pf_bytes[i], blockIdx.x, gridDim.x, lane);
   const int task = blockIdx.x * kW + warp;
   const int grp = task / (8 * NT), m = task % (8 * NT);
   const bool live = task < r.G * 8 * NT;
@@ -958,6 +986,11 @@ qlin_status launch_gemv_tc(const PackedView& v, const __half* scales, const __ha
     r.M = M;
     r.K = v.K;
     r.G = a.p.G;
+    r.pf[0] = v.codes;
+    r.pf_bytes[0] = (size_t)v.N * (size_t)v.row_bytes_uniform;
+    r.pf[1] = scales;
+    r.pf[2] = zeros;
+    r.pf_bytes[1] = r.pf_bytes[2] = (size_t)v.N * (size_t)a.p.G * 2;
   }
   switch (B) {
     case 3: return launch_tc_bits<3>(a, r, st);
