@@ -266,6 +266,23 @@ def test_gemv_m1_shapes(bits, N, K):
     _gemv_case(w, a, what=f"b{bits} N{N} K{K} M1")
 
 
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("N,K", [(2368, 1280), (2516, 1408), (2900, 2560), (2960, 1408), (3108, 1280), (9728, 1280)])
+def test_gemv_m1_integer_last_tile(bits, N, K):
+    """The integer M = 1 kernel with a CTA's last 16-row tile full (2368 rows: 16 a CTA) or holding 1,
+    3, 4 or 5 rows (the rows past the CTA's share read its last row and store nothing), including an
+    odd number of groups (K = 1408: the last group pair has one group), against the oracle on every
+    row."""
+    w = _rand_weight(N, K, bits, seed=7 * N + bits)
+    a = W.draw_activation(1, K, seed=N + 3).to(DEV)
+    d, packed = packed_on_device(w)
+    assert Q.qlin_gemv_plan(d, 1)["kernel"] == 3
+    y = Q.qlin_gemv(d, packed, w.scales, w.zeros, a.sign_bits, a.x)
+    torch.cuda.synchronize()
+    assert_close(y, oracle_rows(w, a), f"b{bits} N{N} K{K} M1")
+    assert_dot_bound(y, w, a, what=f"b{bits} N{N} K{K} M1")
+
+
 @pytest.mark.parametrize("bits", [3, 4, 6, 8])
 @pytest.mark.parametrize("N,K", [(4737, 1280), (5000, 1024), (6000, 1536), (4800, 4096), (5000, 128), (9728, 384)])
 def test_gemv_m1_tall_shapes(bits, N, K):
