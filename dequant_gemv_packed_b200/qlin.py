@@ -53,6 +53,8 @@ class Desc:
             ptr = ctypes.addressof(self._bb)
         self.block_bits = None if self._bb is None else list(self._bb.raw)
         self.c = _Desc(self.N, self.K, self.bits, ptr)
+        self._byref = ctypes.byref(self.c)
+        self._ws = {}  # (entry point, M) -> workspace bytes: a pure function of the descriptor and M
 
     @classmethod
     def of(cls, w) -> "Desc":
@@ -60,7 +62,7 @@ class Desc:
         return cls(w.N, w.K, w.bits, w.block_bits)
 
     def ref(self):
-        return ctypes.byref(self.c)
+        return self._byref
 
 
 _lib = None
@@ -112,8 +114,13 @@ def _check(status: int, what: str) -> None:
         raise QlinError(status, what)
 
 
-def _stream(stream) -> int:
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream, like: torch.Tensor = None) -> int:
     if stream is None:
+        if _raw_stream is not None and like is not None and like.is_cuda:
+            return _raw_stream(like.device.index)  # the current stream's handle, without a Stream object
         return torch.cuda.current_stream().cuda_stream
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
@@ -265,14 +272,16 @@ def _linear(fn, what, ws_fn, desc, packed, scales, zeros, sign_bits, x, y, works
         raise ValueError("x.shape[1] != desc.K")
     if y is None:
         y = _alloc((M, desc.N), torch.float16, x)
-    ws = ws_fn(desc, M)
+    ws = desc._ws.get((what, M))
+    if ws is None:
+        ws = desc._ws[(what, M)] = ws_fn(desc, M)
     if workspace is None and ws:
         workspace = _alloc((ws,), torch.uint8, x)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(fn(desc.ref(), _dev(packed, torch.uint8, "packed"), _dev(scales, torch.float16, "scales"),
               _dev(zeros, torch.float16, "zeros"), _dev(sign_bits, torch.int32, "sign_bits"),
-              _dev(x, torch.float16, "x"), _dev(y, torch.float16, "y"), M, ws_ptr, ws_len, _stream(stream)), what)
+              _dev(x, torch.float16, "x"), _dev(y, torch.float16, "y"), M, ws_ptr, ws_len, _stream(stream, x)), what)
     return y
 
 
