@@ -701,7 +701,15 @@ qlin_status launch_gemm_rotated(const PackedView& v, const __half* scales, const
   a.m_tiles = (M + a.BN - 1) / a.BN;
   a.n_tiles = (v.N + kBMw - 1) / kBMw;
   a.KB = v.K / kBK;
-  a.stream_k = flags != nullptr ? 1 : 0;
+  // Stream-K unless the tiles alone already fill at least half of the SMs and
+  // a split tile's partial sum would be large (BN >= 192: a split costs the
+  // owner ~4 us of waiting for and adding 96-128 KB): then one CTA per tile
+  // (prefill M = 256: 33.0 instead of 35.3 us; at M = 32 or 512 stream-K wins).
+  {
+    const long long tiles = (long long)a.m_tiles * a.n_tiles;
+    const bool per_tile = a.BN >= 192 && tiles <= kSms && 2 * tiles >= kSms;
+    a.stream_k = (flags != nullptr && !per_tile) ? 1 : 0;
+  }
   a.part_cols = (a.BN + 31) & ~31;
   a.flags = flags;
   a.partials = partials;
