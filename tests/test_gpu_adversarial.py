@@ -47,7 +47,8 @@ def _run(w, a, M):
     return y
 
 
-PATHS = [(1, 3), (1, 4), (1, 6), (1, 8), (4, 3), (4, 8), (16, 4), (16, 6), (256, 6), (256, 0)]
+PATHS = [(1, 3), (1, 4), (1, 6), (1, 8), (2, 6), (4, 3), (4, 8), (9, 3), (16, 4), (16, 6), (32, 0), (64, 8),
+         (256, 6), (256, 0)]
 
 
 def _bb(bits, n):
