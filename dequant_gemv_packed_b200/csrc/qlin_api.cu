@@ -262,4 +262,31 @@ qlin_status qlin_gemm(const qlin_desc* d, const void* packed, const uint16_t* sc
                      workspace, reinterpret_cast<cudaStream_t>(st));
 }
 
+qlin_status qlin_linear_host(const qlin_desc* d, const void* packed, const uint16_t* scales,
+                             const uint16_t* zeros, const uint32_t* sign_bits, const uint16_t* x_host,
+                             uint16_t* y_host, uint16_t* x_dev, uint16_t* y_dev, int32_t M, void* workspace,
+                             size_t workspace_bytes, qlin_stream_t st) {
+  if (!x_host || !y_host) return QLIN_ERR_INVALID_ARG;
+  qlin_status r = check_linear(d, packed, scales, zeros, sign_bits, x_dev, y_dev);
+  if (r != QLIN_OK) return r;
+  if (M < 1) return QLIN_ERR_SHAPE;
+  // every check before the first enqueue: an error enqueues nothing
+  const bool gemv = M <= 16;
+  const size_t ws = gemv ? gemv_workspace_bytes(d->bits, d->N, d->K, M) : gemm_workspace_bytes(M, d->K);
+  if (ws && (!workspace || workspace_bytes < ws)) return QLIN_ERR_WORKSPACE;
+  if (ws && !aligned16(workspace)) return QLIN_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(st);
+  cudaError_t e = cudaMemcpyAsync(x_dev, x_host, (size_t)M * (size_t)d->K * 2, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return record_cuda(e);
+  const PackedView v = make_view(d, packed);
+  const __half* xs = reinterpret_cast<const __half*>(x_dev);
+  __half* ys = reinterpret_cast<__half*>(y_dev);
+  r = gemv ? launch_gemv(v, reinterpret_cast<const __half*>(scales), reinterpret_cast<const __half*>(zeros),
+                         sign_bits, xs, ys, M, workspace, s)
+           : launch_gemm(v, reinterpret_cast<const __half*>(scales), reinterpret_cast<const __half*>(zeros),
+                         sign_bits, xs, ys, M, workspace, s);
+  if (r != QLIN_OK) return r;
+  return record_cuda(cudaMemcpyAsync(y_host, y_dev, (size_t)M * (size_t)d->N * 2, cudaMemcpyDeviceToHost, s));
+}
+
 }  // extern "C"

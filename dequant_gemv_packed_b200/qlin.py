@@ -23,7 +23,7 @@ EXPORTED = (
     "qlin_status_string", "qlin_last_cuda_error", "qlin_packed_bytes", "qlin_code_bytes", "qlin_pack",
     "qlin_unpack", "qlin_dequant", "qlin_rht", "qlin_gemv_workspace_bytes", "qlin_gemv",
     "qlin_gemm_workspace_bytes", "qlin_gemm", "qlin_device_error", "qlin_gemm_noalloc", "qlin_set_overlap",
-    "qlin_quantize_rtn", "qlin_gemv_plan", "qlin_gptq_workspace_bytes", "qlin_quantize_gptq",
+    "qlin_quantize_rtn", "qlin_gemv_plan", "qlin_gptq_workspace_bytes", "qlin_quantize_gptq", "qlin_linear_host",
 )
 
 
@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
     L.qlin_gemv.argtypes, L.qlin_gemv.restype = lin, ctypes.c_int
     L.qlin_gemm.argtypes, L.qlin_gemm.restype = lin, ctypes.c_int
     L.qlin_gemm_noalloc.argtypes, L.qlin_gemm_noalloc.restype = [vp, vp, vp, vp, vp, vp, vp, i32, vp], ctypes.c_int
+    L.qlin_linear_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
+    L.qlin_linear_host.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -299,6 +301,42 @@ def qlin_linear(desc: Desc, packed, scales, zeros, sign_bits, x, y=None, workspa
     """qlin_gemv for M <= 16, qlin_gemm otherwise."""
     f = qlin_gemv if x.shape[0] <= 16 else qlin_gemm
     return f(desc, packed, scales, zeros, sign_bits, x, y, workspace, stream)
+
+
+def _host(t: torch.Tensor, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise TypeError(f"{name} must be a host tensor")
+    if t.dtype != torch.float16:
+        raise TypeError(f"{name} must be torch.float16, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def qlin_linear_host(desc: Desc, packed, scales, zeros, sign_bits, x_host, y_host, x_dev, y_dev,
+                     workspace=None, stream=None) -> torch.Tensor:
+    """The layer on host activations in one call (x_host [M, K] and y_host [M, N]
+    fp16 host tensors, pinned for asynchronous copies; x_dev / y_dev device
+    staging tensors of the same shapes); returns y_host, valid once the stream
+    has passed the call."""
+    M, K = x_host.shape
+    if K != desc.K or tuple(y_host.shape) != (M, desc.N) or tuple(x_dev.shape) != (M, K) \
+            or tuple(y_dev.shape) != (M, desc.N):
+        raise ValueError("shapes: x_host/x_dev [M, K], y_host/y_dev [M, N]")
+    what = "qlin_gemv" if M <= 16 else "qlin_gemm"
+    ws = desc._ws.get((what, M))
+    if ws is None:
+        ws = desc._ws[(what, M)] = (qlin_gemv_workspace_bytes if M <= 16 else qlin_gemm_workspace_bytes)(desc, M)
+    if workspace is None and ws:
+        workspace = _alloc((ws,), torch.uint8, x_dev)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().qlin_linear_host(desc.ref(), _dev(packed, torch.uint8, "packed"), _dev(scales, torch.float16, "scales"),
+                                  _dev(zeros, torch.float16, "zeros"), _dev(sign_bits, torch.int32, "sign_bits"),
+                                  _host(x_host, "x_host"), _host(y_host, "y_host"), _dev(x_dev, torch.float16, "x_dev"),
+                                  _dev(y_dev, torch.float16, "y_dev"), M, ws_ptr, ws_len, _stream(stream, x_dev)),
+           "qlin_linear_host")
+    return y_host
 
 
 def algorithmic_bytes(desc: Desc) -> int:

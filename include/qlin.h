@@ -345,6 +345,25 @@ qlin_status qlin_gemm_noalloc(const qlin_desc* desc, const void* packed, const u
                               const uint16_t* zeros, const uint32_t* sign_bits, const uint16_t* x,
                               uint16_t* y, int32_t M, qlin_stream_t stream);
 
+/* The layer for activations that live in host memory, in one call: copies x
+ * in, runs qlin_gemv (M <= 16) or qlin_gemm (M > 16) on it, and copies y back,
+ * all enqueued on `stream` in that order (three asynchronous operations, one
+ * per copy and the layer's kernels).  The pages have no counterpart; this is
+ * a library convenience for a caller whose activations are on the host.
+ *   x_host : host fp16 [M][K];  y_host : host fp16 [M][N].  Both must stay
+ *            valid until the stream has passed the copies; page-locked
+ *            (pinned) memory keeps the copies asynchronous.
+ *   x_dev, y_dev : device fp16 [M][K] and [M][N] staging buffers (16-byte
+ *            aligned), overwritten;
+ *   workspace : as qlin_gemv (M <= 16) or qlin_gemm (M > 16) need it.
+ *   Result: y_host holds the same bits as the device call would write into
+ *   y_dev.  Every argument is checked before the first copy is enqueued, so an
+ *   error enqueues nothing. */
+qlin_status qlin_linear_host(const qlin_desc* desc, const void* packed, const uint16_t* scales,
+                             const uint16_t* zeros, const uint32_t* sign_bits, const uint16_t* x_host,
+                             uint16_t* y_host, uint16_t* x_dev, uint16_t* y_dev, int32_t M, void* workspace,
+                             size_t workspace_bytes, qlin_stream_t stream);
+
 /* Reads and clears the device-side error word (0 = no error).  Kernels that
  * wait on shared-memory barriers bound every wait; a wait that gives up sets a
  * bit here instead of hanging (the call's output is then invalid): bits 0-7

@@ -228,3 +228,27 @@ def test_gemv_plan_validation(lib):
     assert lib.qlin_gemv_plan(Q.Desc(64, 128, 4).ref(), 1, None) == -1
     assert lib.qlin_gemv_plan(Q.Desc(64, 100, 4).ref(), 1, info) == -3
     assert lib.qlin_gemv_plan(None, 1, info) == -1
+
+
+def test_linear_host_validation_returns_before_enqueue(lib):
+    """qlin_linear_host checks every argument before its first copy: missing host
+    buffers, a missing or small workspace and misaligned staging buffers are
+    reported without a CUDA call (the pointers below are never dereferenced).
+    Status codes: -1 invalid argument, -3 shape, -4 alignment, -6 workspace."""
+    d = Q.Desc(2560, 9728, 3)
+    dev = [ctypes.c_void_p(0x100000 * (i + 1)) for i in range(7)]  # 16-byte aligned stand-ins
+    host = ctypes.c_void_p(0x7F0000000000)
+
+    def call(M, x_host, y_host, x_dev, ws, ws_len):
+        return lib.qlin_linear_host(d.ref(), dev[0], dev[1], dev[2], dev[3], x_host, y_host, x_dev, dev[4], M, ws,
+                                    ws_len, None)
+
+    assert call(1, None, host, dev[5], None, 0) == -1
+    assert call(1, host, None, dev[5], None, 0) == -1
+    assert call(0, host, host, dev[5], None, 0) == -3
+    assert call(1, host, host, ctypes.c_void_p(0x100002), None, 0) == -4
+    need = Q.qlin_gemv_workspace_bytes(d, 4)
+    assert need > 0
+    assert call(4, host, host, dev[5], None, 0) == -6
+    assert call(4, host, host, dev[5], dev[6], need - 16) == -6
+    assert call(32, host, host, dev[5], dev[6], 1024) == -6

@@ -449,6 +449,26 @@ def test_gemm_matches_gemv_at_m16():
     assert_close(y2, ref, "gemm")
 
 
+@pytest.mark.parametrize("M,bits", [(1, 4), (1, 3), (4, 6), (32, 0)])
+def test_linear_host_matches_device_call(M, bits):
+    """qlin_linear_host (x from pinned host memory, y back to it, one call) gives
+    the bits the device call gives, and both match the oracle."""
+    N, K = 512, 1280
+    w = _rand_weight(N, K, bits, seed=90 + M + bits, block_bits=[6, 8, 4, 3, 8, 6, 8, 4] if bits == 0 else None)
+    a = W.draw_activation(M, K, seed=91 + M).to(DEV)
+    d, packed = packed_on_device(w)
+    fn = Q.qlin_gemv if M <= 16 else Q.qlin_gemm
+    y_dev = fn(d, packed, w.scales, w.zeros, a.sign_bits, a.x)
+    xh = a.x.cpu().pin_memory()
+    yh = torch.full((M, N), float("nan"), dtype=torch.float16).pin_memory()
+    xd = torch.empty_like(a.x)
+    yd = torch.empty(M, N, dtype=torch.float16, device=DEV)
+    Q.qlin_linear_host(d, packed, w.scales, w.zeros, a.sign_bits, xh, yh, xd, yd)
+    torch.cuda.synchronize()
+    assert torch.equal(yh.view(torch.int16), y_dev.cpu().view(torch.int16))
+    assert_close(yh, oracle_rows(w, a), f"linear_host M{M} b{bits}")
+
+
 def test_zz_no_device_errors():
     """No bounded wait in any kernel gave up during the tests above."""
     torch.cuda.synchronize()
