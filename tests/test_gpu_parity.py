@@ -267,12 +267,14 @@ def test_gemv_m1_shapes(bits, N, K):
 
 
 @pytest.mark.parametrize("bits", [4, 8])
-@pytest.mark.parametrize("N,K", [(2368, 1280), (2516, 1408), (2900, 2560), (2960, 1408), (3108, 1280), (9728, 1280)])
+@pytest.mark.parametrize("N,K", [(2368, 1280), (2516, 1408), (2900, 2560), (2960, 1408), (3108, 1280), (9728, 1280),
+                                 (2368, 3072), (4736, 2816), (4736, 2304)])
 def test_gemv_m1_integer_last_tile(bits, N, K):
     """The integer M = 1 kernel with a CTA's last 16-row tile full (2368 rows: 16 a CTA) or holding 1,
     3, 4 or 5 rows (the rows past the CTA's share read its last row and store nothing), including an
-    odd number of groups (K = 1408: the last group pair has one group), against the oracle on every
-    row."""
+    odd number of groups (K = 1408: the last group pair has one group), and 17 to 24 groups (K = 2304,
+    2560, 2816, 3072: the second rotation round runs beside the main loop), against the oracle on
+    every row."""
     w = _rand_weight(N, K, bits, seed=7 * N + bits)
     a = W.draw_activation(1, K, seed=N + 3).to(DEV)
     d, packed = packed_on_device(w)
