@@ -273,7 +273,7 @@ def test_gemv_m1_integer_last_tile(bits, N, K):
     """The integer M = 1 kernel with a CTA's last 16-row tile full (2368 rows: 16 a CTA) or holding 1,
     3, 4 or 5 rows (the rows past the CTA's share read its last row and store nothing), including an
     odd number of groups (K = 1408: the last group pair has one group), and 17 to 24 groups (K = 2304,
-    2560, 2816, 3072: the second rotation round runs beside the main loop), against the oracle on
+    2560, 2816, 3072: the groups past the sixteenth take a second rotation round), against the oracle on
     every row."""
     w = _rand_weight(N, K, bits, seed=7 * N + bits)
     a = W.draw_activation(1, K, seed=N + 3).to(DEV)
