@@ -285,6 +285,23 @@ def test_gemv_m1_integer_last_tile(bits, N, K):
     assert_dot_bound(y, w, a, what=f"b{bits} N{N} K{K} M1")
 
 
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("N,K", [(147, 2560), (1337, 2560), (2368, 5120), (1184, 8192), (296, 9728)])
+def test_gemv_m1_integer_rotation_rounds(bits, N, K):
+    """The integer M = 1 kernel when its 16 warps rotate x in several rounds:
+    20 groups (four warps take a second block; on 148 CTAs and on an odd grid
+    of 147), 40, 64 and 76 groups (three to five rounds), against the oracle on
+    every row."""
+    w = _rand_weight(N, K, bits, seed=11 * N + bits)
+    a = W.draw_activation(1, K, seed=N + 5).to(DEV)
+    d, packed = packed_on_device(w)
+    assert Q.qlin_gemv_plan(d, 1)["kernel"] == 3
+    y = Q.qlin_gemv(d, packed, w.scales, w.zeros, a.sign_bits, a.x)
+    torch.cuda.synchronize()
+    assert_close(y, oracle_rows(w, a), f"b{bits} N{N} K{K} M1")
+    assert_dot_bound(y, w, a, what=f"b{bits} N{N} K{K} M1")
+
+
 @pytest.mark.parametrize("bits", [3, 4, 6, 8])
 @pytest.mark.parametrize("N,K", [(4737, 1280), (5000, 1024), (6000, 1536), (4800, 4096), (5000, 128), (9728, 384)])
 def test_gemv_m1_tall_shapes(bits, N, K):
