@@ -584,14 +584,25 @@ PER_CONFIG = (("tiny", 4000, 20), ("down1", 4000, 20), ("down4", 2000, 20), ("do
               ("prefill1024", 400, 10), ("prefill2048", 200, 10), ("quantize", 1000, 20), ("gptq", 5, 3))
 
 
+L2_POLICY = {
+    "gemv": "inputs larger than L2: consecutive timed calls rotate over packed-weight copies totalling more than 2x L2",
+    "gemm": "inputs larger than L2: consecutive timed calls rotate over packed-weight copies totalling more than 2x L2",
+    "stack": "inputs larger than L2: one step streams every layer's packed weight (3.2 GB)",
+    "quantize": "inputs larger than L2: consecutive timed calls rotate over fp16 weight copies totalling more than 2x L2",
+    "gptq": "inputs larger than L2: the fp16 weight and its fp32 working copy",
+}
+
+
 def workload_config(case, world: int) -> dict:
-    """What the workload is (identical in both arms): shapes, widths, inputs."""
+    """What the workload is (identical in both arms): shapes, widths, inputs,
+    and how the timed region keeps L2 from serving repeated inputs."""
     bits = getattr(case, "bits", None)
     return {"workload": case.desc_text, "M": case.M, "K": case.K, "N": case.N, "group": 128,
             "bits": ("mixed int6/int8" if bits == 0 else bits) if case.kind != "stack" else "int6 + int8 lm_head",
             "parallelism": f"replicas x{world}",
             "inputs": "seeded synthetic: weights N(0,0.02) with 0.1% x20 outliers, RTN g128 fp16 scale/zero; "
-                      "activations N(0,1) fp16; random signs"}
+                      "activations N(0,1) fp16; random signs",
+            "l2": L2_POLICY[case.kind]}
 
 
 def roofline_of(case, ms_step: float, peaks: dict) -> dict:
