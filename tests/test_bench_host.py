@@ -20,6 +20,18 @@ def test_workload_tables_cover_every_kind():
             assert os.path.exists(os.path.join(csrc, f)), f
 
 
+def test_workload_config_for_every_workload():
+    """The config dict (identical in both arms) names the workload and how the
+    timed region keeps L2 from serving repeated inputs, for every workload."""
+    from types import SimpleNamespace
+    for name, (desc, kind, p) in bench.WORKLOADS.items():
+        case = SimpleNamespace(desc_text=desc, M=p.get("M", 1), K=2560, N=9728, bits=4, kind=kind)
+        cfg = bench.workload_config(case, 1)
+        assert cfg["workload"] == desc and cfg["parallelism"] == "replicas x1"
+        assert cfg["l2"].startswith("inputs larger than L2"), name
+        json.dumps(cfg)
+
+
 def test_source_hash_follows_the_kernel_file(tmp_path, monkeypatch):
     """A kind's hash covers its own .cu file and the shared headers, not the
     other kernels' files; the whole-directory hash covers everything."""
